@@ -1,0 +1,275 @@
+"""Pins for the CPU oracle: each test ties the oracle to something other than
+itself (a library routine on a differently built input, a closed form, brute
+force, or a value printed on the pages), so that a dropped term, a wrong sign
+or index, or a transposed operand in the oracle fails at least one of them.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+from sparse_approximate_attention_b200 import workloads as W
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _small(la=16, blocks=(24, 20, 32, 17), lq=9, lp=5, hq=4, hkv=2, d=16,
+           seed=7, scale=None):
+    lay = oracle.make_layout(len(blocks) // 2, la, list(blocks), lq, lp, hq, hkv,
+                             d, scale)
+    g = torch.Generator().manual_seed(seed)
+    n = lay.n
+    Q = torch.randn(n, hq, d, generator=g, dtype=torch.float64)
+    K = torch.randn(n, hkv, d, generator=g, dtype=torch.float64)
+    Vv = torch.randn(n, hkv, d, generator=g, dtype=torch.float64)
+    return lay, Q, K, Vv
+
+
+def _sdpa_causal(Q, K, V, scale):
+    """Library dense causal attention, fp64: (o [n,Hq,d], lse [Hq,n])."""
+    n, hq, d = Q.shape
+    G = hq // K.shape[1]
+    q = Q.permute(1, 0, 2)
+    k = K.repeat_interleave(G, dim=1).permute(1, 0, 2)
+    v = V.repeat_interleave(G, dim=1).permute(1, 0, 2)
+    o = F.scaled_dot_product_attention(q[None], k[None], v[None], is_causal=True,
+                                       scale=scale)[0]
+    z = scale * (q @ k.transpose(1, 2))
+    z = z.masked_fill(torch.triu(torch.ones(n, n, dtype=torch.bool), 1), -math.inf)
+    return o.permute(1, 0, 2).numpy(), torch.logsumexp(z, dim=-1).numpy()
+
+
+# ---------------------------------------------------------------- selection
+def test_top_lp_brute_force_dominance():
+    """Among all k-subsets exactly one satisfies 'every kept score beats every
+    dropped one, equal scores keep the lower index'; the oracle returns it."""
+    rng = np.random.default_rng(3)
+    for trial in range(40):
+        L = int(rng.integers(1, 9))
+        k = int(rng.integers(0, L + 1))
+        s = rng.choice([-1.0, 0.0, 0.5, 2.0], size=L) if trial % 2 else rng.normal(size=L)
+        ok = []
+        for sub in itertools.combinations(range(L), k):
+            keep = set(sub)
+            good = all((s[i] > s[j]) or (s[i] == s[j] and i < j)
+                       for i in keep for j in range(L) if j not in keep)
+            if good:
+                ok.append(list(sub))
+        assert len(ok) == 1
+        assert oracle.top_lp(s, k).tolist() == ok[0]
+
+
+def test_top_lp_matches_library_topk_on_distinct_values():
+    g = torch.Generator().manual_seed(11)
+    s = torch.randn(5000, generator=g, dtype=torch.float64)
+    for k in (0, 1, 17, 2500, 5000):
+        ref = torch.sort(torch.topk(s, k).indices).values.numpy() if k else np.zeros(0)
+        assert np.array_equal(oracle.top_lp(s.numpy(), k), ref)
+
+
+def test_top_lp_signed_zero_and_clamp():
+    s = np.array([-0.0, 0.0, -0.0, 1.0], dtype=np.float32)
+    assert oracle.top_lp(s, 2).tolist() == [0, 3]       # -0 == +0, lower index wins
+    assert oracle.top_lp(s, 10).tolist() == [0, 1, 2, 3]  # lp > L clamps
+
+
+# ---------------------------------------------------------------- scoring
+def test_scores_closed_form_axis_queries():
+    """Every query-block query equal to c*e_a makes the score of key j equal
+    to lq * G * scale * c * K[j, kv, a]."""
+    lay, Q, K, Vv = _small()
+    a, c = 3, 0.75
+    Q[lay.query_start:] = 0.0
+    Q[lay.query_start:, :, a] = c
+    for h in range(lay.V - 1):
+        s = oracle.importance_scores(lay, Q, K, h)
+        s0, L = lay.block_starts[h], lay.block_lens[h]
+        for kv in range(lay.num_kv_heads):
+            want = lay.query_len * lay.group * lay.scale * c * K[s0:s0 + L, kv, a].numpy()
+            np.testing.assert_allclose(s[kv], want, rtol=1e-12, atol=1e-12)
+
+
+def test_scores_depend_only_on_own_kv_group():
+    """Changing the queries of the other KV head's group leaves scores alone;
+    changing a query of the own group changes them."""
+    lay, Q, K, Vv = _small()
+    s = oracle.importance_scores(lay, Q, K, 1)
+    Q2 = Q.clone()
+    Q2[lay.query_start:, lay.group:, :] += 1.0          # group of kv head 1
+    s2 = oracle.importance_scores(lay, Q2, K, 1)
+    np.testing.assert_array_equal(s[0], s2[0])
+    assert not np.allclose(s[1], s2[1])
+
+
+def test_planted_needles_are_selected():
+    wl = W.workloads()["tiny"]
+    inp = W.make_inputs(wl)
+    lay = oracle.make_layout(wl.num_hosts, wl.anchor_len, wl.block_lens, wl.query_len,
+                             wl.lp, wl.num_q_heads, wl.num_kv_heads, wl.head_dim)
+    scores, idx = oracle.compress(lay, inp["Q"], inp["K"])
+    needles = inp["needle_positions"].numpy()
+    for h in range(lay.V - 1):
+        chosen = set((lay.block_starts[h] + idx[h][0]).tolist())
+        mine = [p for p in needles if lay.block_starts[h] <= p < lay.block_starts[h] + lay.block_lens[h]]
+        assert len(mine) == 8 and set(mine) <= chosen
+
+
+# ---------------------------------------------------------------- attention
+def test_attend_single_key_and_uniform_closed_form():
+    rng = np.random.default_rng(0)
+    q, k, v = rng.normal(size=(3, 8)), rng.normal(size=(1, 8)), rng.normal(size=(1, 8))
+    o, lse = oracle.attend(q, k, v, 0.5)
+    np.testing.assert_allclose(lse, 0.5 * (q @ k.T)[:, 0], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(o, np.repeat(v, 3, 0), rtol=0, atol=1e-14)
+    k5 = np.repeat(k, 5, 0)
+    v5 = rng.normal(size=(5, 8))
+    o, lse = oracle.attend(q, k5, v5, 0.5)
+    np.testing.assert_allclose(lse, 0.5 * (q @ k.T)[:, 0] + math.log(5), atol=1e-13)
+    np.testing.assert_allclose(o, np.repeat(v5.mean(0, keepdims=True), 3, 0), atol=1e-13)
+
+
+def test_dense_causal_when_passing_is_full_block():
+    """lp >= every block length: the passing blocks are whole earlier blocks,
+    so the layer is exact dense causal attention (library SDPA)."""
+    lay, Q, K, Vv = _small(lp=64)
+    out = oracle.layer_fwd(lay, Q, K, Vv)
+    o_ref, lse_ref = _sdpa_causal(Q, K, Vv, lay.scale)
+    np.testing.assert_allclose(out["O"], o_ref, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(out["lse"], lse_ref, rtol=0, atol=1e-12)
+
+
+def test_dense_causal_unequal_blocks_and_custom_scale():
+    lay, Q, K, Vv = _small(la=5, blocks=(7, 31, 3, 12, 20, 1), lq=4, lp=40, scale=0.3)
+    out = oracle.layer_fwd(lay, Q, K, Vv)
+    o_ref, lse_ref = _sdpa_causal(Q, K, Vv, 0.3)
+    np.testing.assert_allclose(out["O"], o_ref, atol=1e-12)
+    np.testing.assert_allclose(out["lse"], lse_ref, atol=1e-12)
+
+
+@pytest.mark.parametrize("lp", [0, 1, 5])
+def test_query_anchor_and_host0_rows_exact_for_any_lp(lp):
+    """Query rows (merged partials), anchor rows and host 0's context rows
+    equal dense causal attention whatever lp is."""
+    lay, Q, K, Vv = _small(lp=lp)
+    out = oracle.layer_fwd(lay, Q, K, Vv)
+    o_ref, lse_ref = _sdpa_causal(Q, K, Vv, lay.scale)
+    exact = list(range(lay.anchor_len)) + \
+        list(range(lay.block_starts[0], lay.block_starts[0] + lay.block_lens[0])) + \
+        list(range(lay.query_start, lay.n))
+    np.testing.assert_allclose(out["O"][exact], o_ref[exact], atol=1e-12)
+    np.testing.assert_allclose(out["lse"][:, exact], lse_ref[:, exact], atol=1e-12)
+    if lp < min(lay.block_lens):   # later hosts really are approximate
+        late = list(range(lay.block_starts[3], lay.block_starts[3] + lay.block_lens[3]))
+        assert np.abs(out["O"][late] - o_ref[late]).max() > 1e-3
+
+
+@pytest.mark.parametrize("la,lp", [(16, 5), (0, 5), (16, 0), (0, 0)])
+def test_context_rows_equal_causal_attention_on_reduced_sequence(la, lp):
+    """Host h's context rows equal library causal attention over the physically
+    built sequence [B_a, passing keys of hosts < h, B^(h)] (covers the
+    'w/o anchor' la=0 and 'w/o passing' lp=0 ablations)."""
+    lay, Q, K, Vv = _small(la=la, lp=lp)
+    out = oracle.layer_fwd(lay, Q, K, Vv)
+    for h in range(lay.V):
+        s0, L = lay.block_starts[h], lay.block_lens[h]
+        for g in range(lay.num_q_heads):
+            kv = g // lay.group
+            keys = np.concatenate([np.arange(la), oracle.passing_positions(lay, out["idx"], h, kv)]).astype(np.int64)
+            pre = len(keys)
+            seq = np.concatenate([keys, np.arange(s0, s0 + L)])
+            q = torch.zeros(len(seq), 1, lay.head_dim, dtype=torch.float64)
+            q[pre:, 0] = Q[s0:s0 + L, g]
+            k = K[torch.as_tensor(seq), kv][:, None]
+            v = Vv[torch.as_tensor(seq), kv][:, None]
+            o_ref, lse_ref = _sdpa_causal(q, k, v, lay.scale)
+            np.testing.assert_allclose(out["O"][s0:s0 + L, g], o_ref[pre:, 0], atol=1e-12)
+            np.testing.assert_allclose(out["lse"][g, s0:s0 + L], lse_ref[0, pre:], atol=1e-12)
+
+
+def test_uniform_keys_pin_key_sets_tie_rule_and_counts():
+    """All keys equal: every score ties, so each passing block is the first
+    lp_eff keys of its block (lower index wins); every row's output is the
+    plain mean of the values it sees and its lse is z + ln(count)."""
+    lay, Q, K, Vv = _small(la=6, blocks=(10, 7, 12, 9), lq=5, lp=4)
+    k0 = torch.randn(lay.head_dim, dtype=torch.float64)
+    K[:] = k0
+    out = oracle.layer_fwd(lay, Q, K, Vv)
+    for r in range(lay.n):
+        kind, h = lay.host_of_row(r)
+        if kind == "context":
+            vis = list(range(lay.anchor_len))
+            for j in range(h):
+                vis += list(range(lay.block_starts[j], lay.block_starts[j] + lay.lp_eff(j)))
+            vis += list(range(lay.block_starts[h], r + 1))
+        else:
+            vis = list(range(r + 1))
+        for g in range(lay.num_q_heads):
+            kv = g // lay.group
+            z = lay.scale * float(Q[r, g] @ k0)
+            assert abs(out["lse"][g, r] - (z + math.log(len(vis)))) < 1e-12
+            np.testing.assert_allclose(out["O"][r, g], Vv[vis, kv].mean(0).numpy(), atol=1e-12)
+
+
+def test_lse_merge_equals_single_pass_over_union():
+    """Merging partials over a random split of the keys equals library
+    attention over all of them (and merging one part is the identity)."""
+    rng = np.random.default_rng(5)
+    q = rng.normal(size=(6, 16))
+    k = rng.normal(size=(40, 16)) * 2
+    v = rng.normal(size=(40, 16))
+    part = rng.integers(0, 4, size=40)
+    parts = [oracle.attend(q, k[part == p], v[part == p], 0.25) for p in range(4)]
+    o, lse = oracle.lse_merge(np.stack([p[0] for p in parts]), np.stack([p[1] for p in parts]))
+    qt, kt, vt = (torch.as_tensor(x)[None, None] for x in (q, k, v))
+    o_ref = F.scaled_dot_product_attention(qt, kt, vt, scale=0.25)[0, 0].numpy()
+    lse_ref = torch.logsumexp(0.25 * torch.as_tensor(q) @ torch.as_tensor(k).T, -1).numpy()
+    np.testing.assert_allclose(o, o_ref, atol=1e-12)
+    np.testing.assert_allclose(lse, lse_ref, atol=1e-12)
+    o1, l1 = oracle.lse_merge(np.stack([parts[0][0]]), np.stack([parts[0][1]]))
+    np.testing.assert_allclose(o1, parts[0][0], atol=1e-15)
+
+
+def test_rows_fwd_matches_full_layer():
+    lay, Q, K, Vv = _small()
+    out = oracle.layer_fwd(lay, Q, K, Vv)
+    rows = [0, 3, 17, 40, 59, 60, 88, lay.query_start, lay.n - 1]
+    heads = [1, 3]
+    r, o, lse = oracle.rows_fwd(lay, Q, K, Vv, out["idx"], rows, heads)
+    np.testing.assert_allclose(o, out["O"][r][:, heads], atol=1e-13)
+    np.testing.assert_allclose(lse, out["lse"][heads][:, r], atol=1e-13)
+
+
+def test_gather_passing_rows():
+    lay, Q, K, Vv = _small()
+    _, idx = oracle.compress(lay, Q, K)
+    Kp, Vp = oracle.gather_passing(lay, K, Vv, idx)
+    off = 0
+    for h in range(lay.V - 1):
+        for t in range(lay.lp_eff(h)):
+            for kv in range(lay.num_kv_heads):
+                src = lay.block_starts[h] + idx[h][kv][t]
+                assert np.array_equal(Kp[off + t, kv], K[src, kv].numpy())
+                assert np.array_equal(Vp[off + t, kv], Vv[src, kv].numpy())
+        off += lay.lp_eff(h)
+    assert off == Kp.shape[0]
+
+
+def test_flops_count_by_enumeration():
+    lay, Q, K, Vv = _small(la=5, blocks=(7, 31, 3, 12), lq=4, lp=6)
+    _, idx = oracle.compress(lay, Q, K)
+    pairs = sum(len(oracle.key_positions(lay, idx, r, 0)) for r in range(lay.n))
+    assert oracle.flops(lay) == 4 * lay.head_dim * lay.num_q_heads * pairs
+
+
+def test_default_hyperparameters_golden():
+    """la = n/64 and lp = n/128, with the pages' own worked numbers."""
+    with open(os.path.join(GOLDEN, "hyperparameters.json")) as f:
+        gold = json.load(f)
+    for case in gold["cases"]:
+        assert list(oracle.default_hyperparameters(case["n"])) == [case["la"], case["lp"]]
