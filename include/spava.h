@@ -1,0 +1,165 @@
+/*
+ * spava.h -- C ABI of the B200 (sm_100a) approximate-attention prefill layer
+ * of Spava / APB-V, with all 2H ZigZag virtual hosts emulated on one GPU.
+ *
+ * Sources (page title and the part of the page that defines each call):
+ *   [SC] "Spava: Accelerating Long-Video Understanding via Sequence-
+ *        Parallelism-aware Approximate Attention" (sciencestack.ai),
+ *        TL;DR and Fig. 2-5 captions.
+ *   [PR] "APB-V: Accelerating Long-Video Understanding via Sequence-
+ *        Parallelism-aware Approximate Attention" (pith.science review):
+ *        "What carries the argument", "Core claim", referee major comment 1,
+ *        minor comment 2, "Axiom & Free-Parameter Ledger".
+ *   [GN] "Technische Samenvatting: APB-V" (gist.science, nl), Methodologie.
+ *
+ * Sequence and layouts.  The token sequence is
+ *     A | B^(0) | B^(1) | ... | B^(V-1) | B_qr,     V = 2H virtual hosts,
+ * an anchor block of la tokens, V context blocks of L_h tokens and a query
+ * block of lq tokens; n = la + sum L_h + lq.  Virtual hosts h and 2H-1-h form
+ * ZigZag pairs on the pages' physical hosts; on one GPU the pairing only
+ * shapes the work order.  All tensors are contiguous, row-major:
+ *     Q, O       [n, Hq,  d]  bf16
+ *     K, V       [n, Hkv, d]  bf16
+ *     lse        [Hq, n]      fp32, natural log of sum exp(scale * q.k)
+ *     qsum       [Hkv, d]     fp32
+ *     scores     [Hkv, S]     fp32, S = sum_{h<V-1} L_h (block h at column
+ *                             start_h - la)
+ *     idx        [V-1, Hkv, lp] int32, block-relative, ascending; entries past
+ *                             lp_eff(h) = min(lp, L_h) are -1
+ *     Kp, Vp     [P, Hkv, d]  bf16, P = sum_{h<V-1} lp_eff(h); block h's rows
+ *                             start at row off_h = sum_{j<h} lp_eff(j)
+ *     O_part     [V, lq, Hq, d] fp32, lse_part [V, Hq, lq] fp32
+ * Query head g reads KV head g / (Hq/Hkv).
+ *
+ * Ownership and errors.  Every tensor pointer is device memory owned by the
+ * caller (the library allocates nothing and keeps no per-call state).  Q, K,
+ * V, Kp, Vp and O must be 16-byte aligned.  Calls are asynchronous on
+ * `stream`.  Argument errors are returned before anything is launched.  A
+ * failed launch returns SPAVA_ERR_CUDA.  The attention kernel bounds every
+ * wait; if one gives up it records a device error word that
+ * spava_device_error() reports (the results of that call are then invalid).
+ */
+#ifndef SPAVA_H_
+#define SPAVA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; 0 is the legacy default stream. */
+typedef struct CUstream_st* spava_stream_t;
+
+typedef enum {
+  SPAVA_OK = 0,
+  SPAVA_ERR_INVALID_ARG = 1, /* bad shape, null or misaligned pointer       */
+  SPAVA_ERR_UNSUPPORTED = 2, /* valid but outside this build's limits       */
+  SPAVA_ERR_WORKSPACE = 3,   /* workspace missing or smaller than required  */
+  SPAVA_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed           */
+  SPAVA_ERR_DEVICE = 5       /* a kernel reported a device-side failure     */
+} spava_status_t;
+
+#define SPAVA_MAX_HOSTS 16   /* H; V = 2H <= 32 virtual hosts */
+
+/* One layer's problem ([SC] Fig. 2 caption; [GN] Context Splitting;
+ * [PR] ledger for la and lp). */
+typedef struct {
+  int32_t num_hosts;         /* H >= 1 physical hosts; V = 2H context blocks */
+  int32_t anchor_len;        /* la >= 0 (0 = the "w/o anchor" ablation)      */
+  const int32_t* block_lens; /* HOST array of 2H lengths, each >= 1          */
+  int32_t query_len;         /* lq >= 1                                       */
+  int32_t lp;                /* passing length >= 0 (0 = "w/o passing");
+                                clamped per block to min(lp, L_h)            */
+  int32_t num_q_heads;       /* Hq >= 1                                       */
+  int32_t num_kv_heads;      /* Hkv >= 1, Hq % Hkv == 0                       */
+  int32_t head_dim;          /* d in {64, 128}                                */
+  float softmax_scale;       /* <= 0 selects 1/sqrt(d)                        */
+} spava_problem_t;
+
+/* Derived sizes, filled by spava_problem_sizes(). */
+typedef struct {
+  int64_t seq_len;        /* n                                               */
+  int64_t query_start;    /* la + sum L_h                                     */
+  int64_t score_cols;     /* S = sum_{h<V-1} L_h                              */
+  int64_t passing_rows;   /* P = sum_{h<V-1} min(lp, L_h)                     */
+  int64_t attn_pairs;     /* visible (row, key) pairs per query head          */
+  double attn_flops;      /* 4 * d * Hq * attn_pairs                          */
+  int64_t attn_tiles;     /* 128-row work items of the attention launch       */
+  size_t workspace_bytes; /* what spava_layer_fwd needs                       */
+} spava_sizes_t;
+
+/* Check a problem and fill its derived sizes.  No CUDA call. */
+spava_status_t spava_problem_sizes(const spava_problem_t* prob, spava_sizes_t* out);
+
+/* Workspace spava_layer_fwd needs (bytes). No CUDA call. */
+spava_status_t spava_workspace_size(const spava_problem_t* prob, size_t* bytes);
+
+/* Step 1, KV importance ([SC] Fig. 5 caption: Q_qr K^(h)T estimates KV
+ * importance; [PR] "What carries the argument").  The score of key j of
+ * block h < V-1 for KV head kv is the sum, over the query block's rows i and
+ * the query heads g of that KV head, of scale * <q_ig, k_j>.  By linearity it
+ * equals <qsum_kv, k_j> with qsum_kv = scale * sum_{i,g} q_ig, which this
+ * call writes to `qsum` and then streams K once to form `scores`. */
+spava_status_t spava_score(const spava_problem_t* prob, const void* Q,
+                           const void* K, float* qsum, float* scores,
+                           spava_stream_t stream);
+
+/* Step 2, top-lp per block and KV head ([PR] "What carries the argument":
+ * each context block compressed to its top-lp key-value pairs).  Larger
+ * score first; equal scores keep the lower index; -0.0 equals +0.0.
+ * Writes `idx` (ascending, -1 padded). */
+spava_status_t spava_select_topk(const spava_problem_t* prob,
+                                 const float* scores, int32_t* idx,
+                                 spava_stream_t stream);
+
+/* Step 3, the passing blocks of all hosts compacted into Kp, Vp: row
+ * off_h + t of KV head kv is key start_h + idx[h][kv][t].  This in-HBM
+ * gather replaces the pages' cross-host all-gather ([PR] "What carries the
+ * argument"; [SC] Fig. 2 caption): host h reads the prefix of off_h rows. */
+spava_status_t spava_gather_passing(const spava_problem_t* prob, const void* K,
+                                    const void* V, const int32_t* idx,
+                                    void* Kp, void* Vp, spava_stream_t stream);
+
+/* Step 4, one launch of causal attention over mixed key segments ([PR]
+ * minor comment 2: Eq. 4 key list [K_a, K_p, K^(h)]; [SC] Fig. 3 fused
+ * context and query forward; Fig. 4 load balancing):
+ *   anchor rows r < la: keys 0..r;
+ *   context rows of host h: A, Kp rows [0, off_h), and B^(h) keys up to r;
+ *   query rows, partial of host h: B^(h) (host 0 also A and B_qr up to r).
+ * Writes O / lse for anchor and context rows, and O_part / lse_part. */
+spava_status_t spava_attn_fwd(const spava_problem_t* prob, const void* Q,
+                              const void* K, const void* V, const void* Kp,
+                              const void* Vp, void* O, float* lse,
+                              float* O_part, float* lse_part,
+                              spava_stream_t stream);
+
+/* Step 5, merge of the query partials ([PR] ledger: lse merging is exact;
+ * [GN] fused context and query forward): lse = log sum_h exp(lse_h),
+ * O = sum_h exp(lse_h - lse) O_h, written to the query rows of O and lse. */
+spava_status_t spava_lse_merge(const spava_problem_t* prob, const float* O_part,
+                               const float* lse_part, void* O, float* lse,
+                               spava_stream_t stream);
+
+/* The whole layer: steps 1-5 in order on `stream`, with every intermediate
+ * carved from `workspace` (device memory, >= spava_workspace_size bytes,
+ * 256-byte aligned).  Outputs O [n, Hq, d] bf16 and lse [Hq, n] fp32. */
+spava_status_t spava_layer_fwd(const spava_problem_t* prob, const void* Q,
+                               const void* K, const void* V, void* O,
+                               float* lse, void* workspace, size_t ws_bytes,
+                               spava_stream_t stream);
+
+/* Device-side error word of the current device (0 = none); synchronizes the
+ * device, then clears the word.  Bit 0: a bounded wait in the attention
+ * kernel gave up. */
+spava_status_t spava_device_error(uint32_t* code);
+
+/* Human-readable name of a status code (static string). */
+const char* spava_status_string(spava_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPAVA_H_ */

@@ -1,0 +1,292 @@
+// Compression stage: query-block sum, KV importance scores, top-lp selection
+// and the passing-buffer gather.  All four are HBM- or latency-bound; none of
+// them is a dense contraction once the score is written in its linear form.
+//
+// "Spava ..." (sciencestack.ai), Fig. 5 caption: Q_qr K^(h)T estimates KV
+// importance and B_c^(h) are the essential KVs; "APB-V ..." (pith.science
+// review), "What carries the argument": each context block is compressed to
+// its top-lp key-value pairs ranked by Q_qr K^T and gathered by later hosts.
+#pragma once
+#include <cooperative_groups.h>
+#include <cuda_bf16.h>
+
+#include "plan.hpp"
+#include "ptx.cuh"
+
+namespace spava {
+
+namespace cg = cooperative_groups;
+
+// ---------------------------------------------------------------------------
+// qsum[kv][c] = scale * sum over query rows i and heads g of KV head kv of
+// Q[qs+i, g, c].  One cluster of kQsumSplit CTAs per KV head: each CTA sums a
+// slice of the (row, head) pairs, then CTA 0 adds the slices in a fixed order
+// through distributed shared memory (deterministic, one launch).
+// ---------------------------------------------------------------------------
+constexpr int kQsumSplit = 8;
+constexpr int kQsumThreads = 256;
+
+template <int D>
+__global__ void __cluster_dims__(kQsumSplit, 1, 1) __launch_bounds__(kQsumThreads)
+    qsum_kernel(const __nv_bfloat16* __restrict__ Q, float* __restrict__ qsum, int64_t qs, int lq,
+                int Hq, int G, float scale) {
+  constexpr int kParts = D / 8;                    // 16-byte chunks per row
+  constexpr int kLanesRows = kQsumThreads / kParts;
+  __shared__ float part[kLanesRows][D];
+  __shared__ float slice[D];
+  cg::cluster_group cluster = cg::this_cluster();
+  const int kv = blockIdx.y;
+  const int rank = static_cast<int>(cluster.block_rank());
+  const int total = lq * G;
+  const int r0 = static_cast<int>((static_cast<int64_t>(total) * rank) / kQsumSplit);
+  const int r1 = static_cast<int>((static_cast<int64_t>(total) * (rank + 1)) / kQsumSplit);
+  const int pc = threadIdx.x % kParts, lr = threadIdx.x / kParts;
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+  for (int rr = r0 + lr; rr < r1; rr += kLanesRows) {
+    const int i = rr / G, g = kv * G + rr % G;
+    const uint4 raw = *reinterpret_cast<const uint4*>(Q + ((qs + i) * Hq + g) * D + pc * 8);
+    const __nv_bfloat16* v = reinterpret_cast<const __nv_bfloat16*>(&raw);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] += __bfloat162float(v[e]);
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) part[lr][pc * 8 + e] = acc[e];
+  __syncthreads();
+  for (int c = threadIdx.x; c < D; c += kQsumThreads) {
+    float s = 0.f;
+    for (int j = 0; j < kLanesRows; ++j) s += part[j][c];
+    slice[c] = s;
+  }
+  cluster.sync();
+  if (rank == 0) {
+    for (int c = threadIdx.x; c < D; c += kQsumThreads) {
+      float s = 0.f;
+      for (int j = 0; j < kQsumSplit; ++j) s += cluster.map_shared_rank(slice, j)[c];
+      qsum[kv * D + c] = s * scale;
+    }
+  }
+  cluster.sync();
+}
+
+// ---------------------------------------------------------------------------
+// scores[kv][j] = <qsum[kv], K[key0 + j, kv, :]> for j < nkeys.  K is streamed
+// once with 16-byte loads; the D/8 lanes that hold one (key, head) row reduce
+// with shuffles.  Grid-stride, kScoreUnroll loads in flight per thread.
+// ---------------------------------------------------------------------------
+constexpr int kScoreThreads = 256;
+constexpr int kScoreUnroll = 4;
+
+template <int D>
+__global__ void __launch_bounds__(kScoreThreads)
+    score_kernel(const __nv_bfloat16* __restrict__ K, const float* __restrict__ qsum,
+                 float* __restrict__ scores, int64_t key0, int64_t nkeys, int Hkv) {
+  extern __shared__ float sq[];
+  constexpr int kParts = D / 8;
+  for (int c = threadIdx.x; c < Hkv * D; c += blockDim.x) sq[c] = qsum[c];
+  __syncthreads();
+  const int64_t cpr = static_cast<int64_t>(Hkv) * kParts;   // chunks per key row
+  const int64_t total = nkeys * cpr;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const uint4* src = reinterpret_cast<const uint4*>(K + key0 * Hkv * D);
+  const int64_t warp_first = static_cast<int64_t>(blockIdx.x) * blockDim.x + (threadIdx.x & ~31);
+  const int lane = threadIdx.x & 31;
+  for (int64_t base = 0; warp_first + base < total; base += stride * kScoreUnroll) {
+    uint4 raw[kScoreUnroll];
+    int64_t ch[kScoreUnroll];
+#pragma unroll
+    for (int u = 0; u < kScoreUnroll; ++u) {
+      ch[u] = warp_first + base + u * stride + lane;
+      raw[u] = ch[u] < total ? __ldcs(src + ch[u]) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < kScoreUnroll; ++u) {
+      const int within = static_cast<int>(ch[u] % cpr);
+      const int kv = within / kParts, pc = within % kParts;
+      const __nv_bfloat16* v = reinterpret_cast<const __nv_bfloat16*>(&raw[u]);
+      const float* q = sq + kv * D + pc * 8;
+      float dot = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) dot = fmaf(__bfloat162float(v[e]), q[e], dot);
+#pragma unroll
+      for (int off = kParts / 2; off >= 1; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+      if (pc == 0 && ch[u] < total) scores[kv * nkeys + ch[u] / cpr] = dot;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// top-lp per (block h < V-1, KV head): MSB-first radix select on
+// order-preserving 32-bit keys finds the lp-th largest key T and how many
+// copies of T to keep; a block-wide scan in index order then writes the kept
+// indices ascending (ties at T keep the lowest indices).
+// ---------------------------------------------------------------------------
+constexpr int kTopkThreads = 1024;
+
+struct TopkParams {
+  int32_t start[kMaxV];   // first score column of block h
+  int32_t L[kMaxV];
+  int32_t k[kMaxV];       // lp_eff(h)
+  int32_t Hkv, lp;
+  int64_t score_cols;
+};
+
+__device__ __forceinline__ uint32_t order_key(float x) {
+  uint32_t u = __float_as_uint(x);
+  if (u == 0x80000000u) u = 0u;   // -0.0 ranks as +0.0
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ uint64_t block_exclusive_scan_u64(uint64_t v, uint64_t* warp_tot) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint64_t x = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    uint64_t y = __shfl_up_sync(0xffffffffu, x, off);
+    if (lane >= off) x += y;
+  }
+  if (lane == 31) warp_tot[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    const int nw = blockDim.x >> 5;
+    uint64_t t = lane < nw ? warp_tot[lane] : 0;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      uint64_t y = __shfl_up_sync(0xffffffffu, t, off);
+      if (lane >= off) t += y;
+    }
+    if (lane < nw) warp_tot[lane] = t;   // inclusive
+  }
+  __syncthreads();
+  const uint64_t before = warp ? warp_tot[warp - 1] : 0;
+  return before + x - v;
+}
+
+__global__ void __launch_bounds__(kTopkThreads)
+    topk_kernel(const float* __restrict__ scores, int32_t* __restrict__ idx, TopkParams p) {
+  __shared__ uint32_t hist[256];
+  __shared__ uint32_t s_prefix, s_k;
+  __shared__ uint64_t warp_tot[32];
+  const int h = blockIdx.x / p.Hkv, kv = blockIdx.x % p.Hkv;
+  const int L = p.L[h], k = p.k[h];
+  const float* s = scores + kv * p.score_cols + p.start[h];
+  int32_t* out = idx + (static_cast<int64_t>(h) * p.Hkv + kv) * p.lp;
+  const int tid = threadIdx.x;
+  for (int t = k + tid; t < p.lp; t += blockDim.x) out[t] = -1;
+  if (k <= 0) return;
+  if (tid == 0) {
+    s_prefix = 0;
+    s_k = static_cast<uint32_t>(k);
+  }
+  uint32_t mask = 0;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = tid; i < 256; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    const uint32_t prefix = s_prefix;
+    for (int i = tid; i < L; i += blockDim.x) {
+      const uint32_t key = order_key(s[i]);
+      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    if (tid < 32) {
+      uint32_t c[8], tot = 0;
+#pragma unroll
+      for (int b = 0; b < 8; ++b) {
+        c[b] = hist[tid * 8 + b];
+        tot += c[b];
+      }
+      uint32_t x = tot;   // inclusive suffix sum over lanes
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        uint32_t y = __shfl_down_sync(0xffffffffu, x, off);
+        if (tid + off < 32) x += y;
+      }
+      uint32_t running = x - tot;   // count in higher bins
+      const uint32_t kk = s_k;
+#pragma unroll
+      for (int b = 7; b >= 0; --b) {
+        if (running < kk && running + c[b] >= kk) {
+          s_prefix = prefix | (static_cast<uint32_t>(tid * 8 + b) << shift);
+          s_k = kk - running;
+        }
+        running += c[b];
+      }
+    }
+    __syncthreads();
+    mask |= 0xFFu << shift;
+  }
+  const uint32_t T = s_prefix;
+  const uint32_t keq = s_k;   // copies of T to keep (>= 1)
+  const int chunk = (L + blockDim.x - 1) / blockDim.x;
+  const int i0 = min(L, tid * chunk), i1 = min(L, i0 + chunk);
+  uint32_t gt = 0, eq = 0;
+  for (int i = i0; i < i1; ++i) {
+    const uint32_t key = order_key(s[i]);
+    gt += key > T;
+    eq += key == T;
+  }
+  const uint64_t pre = block_exclusive_scan_u64((static_cast<uint64_t>(eq) << 32) | gt, warp_tot);
+  uint32_t gt_pre = static_cast<uint32_t>(pre), eq_pre = static_cast<uint32_t>(pre >> 32);
+  for (int i = i0; i < i1; ++i) {
+    const uint32_t key = order_key(s[i]);
+    if (key > T) {
+      out[gt_pre + min(eq_pre, keq)] = i;
+      ++gt_pre;
+    } else if (key == T) {
+      if (eq_pre < keq) out[gt_pre + eq_pre] = i;
+      ++eq_pre;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Kp/Vp[off_h + t, kv, :] = K/V[start_h + idx[h][kv][t], kv, :].  One thread
+// per 16-byte chunk; an index outside its block writes zeros and raises bit 1
+// of the device error word instead of reading out of bounds.
+// ---------------------------------------------------------------------------
+constexpr unsigned int kErrBadIndex = 2u;
+
+struct GatherParams {
+  int32_t start[kMaxV];
+  int32_t L[kMaxV];
+  int32_t poff[kMaxV + 1];
+  int32_t nblocks;   // V - 1
+  int32_t Hkv, lp;
+  int64_t rows;      // passing rows
+};
+
+template <int D>
+__global__ void __launch_bounds__(256)
+    gather_kernel(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restrict__ V,
+                  const int32_t* __restrict__ idx, __nv_bfloat16* __restrict__ Kp,
+                  __nv_bfloat16* __restrict__ Vp, GatherParams p) {
+  constexpr int kParts = D / 8;
+  const int64_t per = p.rows * p.Hkv * kParts;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; c < 2 * per;
+       c += stride) {
+    const int which = c >= per;
+    const int64_t cc = c - which * per;
+    const int pc = static_cast<int>(cc % kParts);
+    const int64_t t2 = cc / kParts;
+    const int kv = static_cast<int>(t2 % p.Hkv);
+    const int64_t prow = t2 / p.Hkv;
+    int h = 0;
+    while (h + 1 < p.nblocks && p.poff[h + 1] <= prow) ++h;
+    const int t = static_cast<int>(prow - p.poff[h]);
+    const int32_t j = idx[(static_cast<int64_t>(h) * p.Hkv + kv) * p.lp + t];
+    uint4 val = make_uint4(0, 0, 0, 0);
+    if (j >= 0 && j < p.L[h]) {
+      const __nv_bfloat16* src = (which ? V : K) +
+                                 ((static_cast<int64_t>(p.start[h]) + j) * p.Hkv + kv) * D + pc * 8;
+      val = *reinterpret_cast<const uint4*>(src);
+    } else if (pc == 0) {
+      atomicOr(&g_device_error, kErrBadIndex);
+    }
+    __nv_bfloat16* dst = (which ? Vp : Kp) + (prow * p.Hkv + kv) * D + pc * 8;
+    *reinterpret_cast<uint4*>(dst) = val;
+  }
+}
+
+}  // namespace spava

@@ -1,0 +1,67 @@
+"""Shared helpers for the parity tests (not collected as tests)."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from sparse_approximate_attention_b200 import workloads as W
+
+# Tolerances of the layer (bf16 inputs, fp32 accumulation): outputs within
+# 2e-2 max-abs, lse within 1e-3; top-lp sets exact except near-ties whose
+# oracle score gap is below 1e-4 of the block's largest |score|.
+O_TOL = 2e-2
+LSE_TOL = 1e-3
+TIE_REL = 1e-4
+
+
+def layout_of(wl: W.Workload) -> oracle.Layout:
+    return oracle.make_layout(wl.num_hosts, wl.anchor_len, wl.block_lens, wl.query_len, wl.lp,
+                              wl.num_q_heads, wl.num_kv_heads, wl.head_dim)
+
+
+def small_workload(name, la, blocks, lq, lp, hq, hkv, d, gen="gaussian", seed=5):
+    return W.Workload(name, num_hosts=len(blocks) // 2, anchor_len=la, block_lens=list(blocks),
+                      query_len=lq, lp=lp, num_q_heads=hq, num_kv_heads=hkv, head_dim=d,
+                      generator=gen, seed=seed)
+
+
+def compare_selection(lay: oracle.Layout, ref_scores: dict, ref_idx: dict, gpu_idx: np.ndarray):
+    """Compare GPU passing indices [V-1, Hkv, lp] with the oracle's.  Returns
+    (tolerated_swaps, affected) where affected[h][kv] is True when the sets
+    differ (only at near-ties, else AssertionError)."""
+    swaps = 0
+    affected = {}
+    for h in range(lay.V - 1):
+        e = lay.lp_eff(h)
+        affected[h] = {}
+        for kv in range(lay.num_kv_heads):
+            g = gpu_idx[h, kv]
+            assert np.all(g[e:] == -1), f"block {h} kv {kv}: padding not -1"
+            gs = g[:e]
+            assert np.all(np.diff(gs) > 0), f"block {h} kv {kv}: indices not ascending/unique"
+            rs = np.asarray(ref_idx[h][kv])
+            diff = set(gs.tolist()) ^ set(rs.tolist())
+            if diff:
+                s = np.asarray(ref_scores[h][kv], dtype=np.float64)
+                tau = np.sort(s)[::-1][e - 1]
+                tol = TIE_REL * np.abs(s).max()
+                bad = [j for j in diff if abs(s[j] - tau) > tol]
+                assert not bad, f"block {h} kv {kv}: non-tie mismatches at {bad[:8]}"
+                swaps += len(set(gs.tolist()) - set(rs.tolist()))
+            affected[h][kv] = bool(diff)
+    return swaps, affected
+
+
+def host_affected(lay, affected, h, kv) -> bool:
+    return any(affected[j][kv] for j in range(min(h, lay.V - 1)))
+
+
+def max_err(a, b) -> float:
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    return float(np.abs(a - b).max()) if a.size else 0.0
+
+
+def to_np(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy() if t.dtype == torch.bfloat16 else t.detach().cpu().numpy()

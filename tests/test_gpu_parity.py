@@ -1,0 +1,226 @@
+"""GPU parity of every stage and of the fused layer against the CPU oracle,
+through the C ABI, on small seeded cases that span several tiles and ragged
+tails (partial anchor / block / query tiles, unequal blocks, la = 0, lp = 0,
+lp >= L_h, G = 1, lq = 1, d = 64 and 128)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sparse_approximate_attention_b200 as spava
+from sparse_approximate_attention_b200 import workloads as W
+
+from helpers import (LSE_TOL, O_TOL, compare_selection, host_affected, layout_of, max_err,
+                     small_workload, to_np)
+
+pytestmark = pytest.mark.gpu
+
+CASES = {
+    "tiny": W.workloads()["tiny"],
+    "ragged_d128": small_workload("ragged_d128", 64, (300, 129, 77, 511), 37, 50, 4, 2, 128),
+    "no_anchor_no_passing": small_workload("no_anchor_no_passing", 0, (130, 200), 5, 0, 2, 1, 128),
+    "dense_unequal_g1": small_workload("dense_unequal_g1", 100, (250, 90, 333, 17, 128, 129), 64,
+                                       400, 2, 2, 128),
+    "pair_lq1_d64": small_workload("pair_lq1_d64", 128, (256, 384), 1, 64, 3, 1, 64),
+    "frames_multi": small_workload("frames_multi", 256, (1024,) * 4, 128, 256, 8, 2, 128,
+                                   gen="frames"),
+    "no_anchor_d64": small_workload("no_anchor_d64", 0, (129, 255, 64, 300, 1, 77), 19, 33, 4, 4, 64),
+}
+
+_cache = {}
+
+
+def _case(name):
+    if name not in _cache:
+        wl = CASES[name]
+        inp = W.make_inputs(wl)
+        lay = layout_of(wl)
+        ref = oracle.layer_fwd(lay, inp["Q"], inp["K"], inp["V"])
+        _cache[name] = (wl, lay, inp, ref)
+    return _cache[name]
+
+
+def _dev(inp):
+    return {k: inp[k].cuda() for k in ("Q", "K", "V")}
+
+
+def _no_device_error():
+    assert spava.device_error() == 0
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_score_stage(name):
+    wl, lay, inp, ref = _case(name)
+    p = spava.Problem.from_workload(wl)
+    d = _dev(inp)
+    qsum, scores = spava.score(p, d["Q"], d["K"])
+    torch.cuda.synchronize()
+    s = to_np(scores)
+    col = 0
+    for h in range(lay.V - 1):
+        r = ref["scores"][h]
+        L = lay.block_lens[h]
+        tol = 1e-5 * np.abs(r).max() + 1e-4
+        assert max_err(s[:, col:col + L], r) <= tol, f"block {h}"
+        col += L
+    assert col == s.shape[1]
+    _no_device_error()
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_topk_stage_on_oracle_scores_is_exact(name):
+    """Both sides decide on the same fp32 scores, so the sets are bit-exact."""
+    wl, lay, inp, ref = _case(name)
+    if wl.lp == 0:
+        pytest.skip("lp = 0 selects nothing")
+    p = spava.Problem.from_workload(wl)
+    s32 = np.concatenate([np.asarray(ref["scores"][h], dtype=np.float32) for h in range(lay.V - 1)], axis=1)
+    idx = to_np(spava.select_topk(p, torch.from_numpy(np.ascontiguousarray(s32)).cuda()))
+    for h in range(lay.V - 1):
+        e = lay.lp_eff(h)
+        for kv in range(lay.num_kv_heads):
+            assert np.array_equal(idx[h, kv, :e], ref["idx"][h][kv]), f"block {h} kv {kv}"
+            assert np.all(idx[h, kv, e:] == -1)
+    _no_device_error()
+
+
+@pytest.mark.parametrize("L,lp,seed", [(1, 1, 0), (7, 3, 1), (1000, 1, 2), (1000, 999, 3),
+                                        (4096, 512, 4), (16384, 2048, 5), (5000, 6000, 6),
+                                        (3000, 64, 7)])
+def test_topk_ties_signed_zero_and_clamp(L, lp, seed):
+    """Planted ties, repeated maxima and +-0.0 against the oracle's rule."""
+    s = W.random_scores(L, 2, seed)
+    p = spava.Problem(1, 0, [L, 1], 1, lp, 2, 2, 64)
+    idx = to_np(spava.select_topk(p, s.cuda().contiguous()))
+    for kv in range(2):
+        want = oracle.top_lp(s[kv].numpy(), lp)
+        e = min(lp, L)
+        assert np.array_equal(idx[0, kv, :e], want)
+        assert np.all(idx[0, kv, e:] == -1)
+    _no_device_error()
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_gather_stage_exact(name):
+    wl, lay, inp, ref = _case(name)
+    if wl.lp == 0:
+        pytest.skip("lp = 0 gathers nothing")
+    p = spava.Problem.from_workload(wl)
+    d = _dev(inp)
+    idx = np.full((lay.V - 1, lay.num_kv_heads, wl.lp), -1, dtype=np.int32)
+    for h in range(lay.V - 1):
+        for kv in range(lay.num_kv_heads):
+            idx[h, kv, :lay.lp_eff(h)] = ref["idx"][h][kv]
+    Kp, Vp = spava.gather_passing(p, d["K"], d["V"], torch.from_numpy(idx).cuda())
+    Kr, Vr = oracle.gather_passing(lay, inp["K"], inp["V"], ref["idx"])
+    assert np.array_equal(to_np(Kp), Kr) and np.array_equal(to_np(Vp), Vr)
+    _no_device_error()
+
+
+def _oracle_passing_dev(lay, inp, ref, hkv, d):
+    Kr, Vr = oracle.gather_passing(lay, inp["K"], inp["V"], ref["idx"])
+    if Kr.shape[0] == 0:
+        return None, None
+    return (torch.from_numpy(Kr).to(torch.bfloat16).cuda().contiguous(),
+            torch.from_numpy(Vr).to(torch.bfloat16).cuda().contiguous())
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_attention_stage(name):
+    """Attention on the oracle's passing buffer: context/anchor rows and the
+    per-host query partials."""
+    wl, lay, inp, ref = _case(name)
+    p = spava.Problem.from_workload(wl)
+    d = _dev(inp)
+    Kp, Vp = _oracle_passing_dev(lay, inp, ref, wl.num_kv_heads, wl.head_dim)
+    O, lse, O_part, lse_part = spava.attn_fwd(p, d["Q"], d["K"], d["V"], Kp, Vp)
+    torch.cuda.synchronize()
+    _no_device_error()
+    qs = lay.query_start
+    assert max_err(to_np(O)[:qs], ref["O"][:qs]) <= O_TOL
+    assert max_err(to_np(lse)[:, :qs], ref["lse"][:, :qs]) <= LSE_TOL
+    assert max_err(to_np(O_part), ref["o_part"]) <= O_TOL
+    assert max_err(to_np(lse_part), ref["lse_part"]) <= LSE_TOL
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_merge_stage(name):
+    wl, lay, inp, ref = _case(name)
+    p = spava.Problem.from_workload(wl)
+    n = lay.n
+    O = torch.zeros(n, wl.num_q_heads, wl.head_dim, dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros(wl.num_q_heads, n, dtype=torch.float32, device="cuda")
+    op = torch.from_numpy(ref["o_part"].astype(np.float32)).cuda().contiguous()
+    lp_ = torch.from_numpy(ref["lse_part"].astype(np.float32)).cuda().contiguous()
+    spava.lse_merge(p, op, lp_, O, lse)
+    torch.cuda.synchronize()
+    qs = lay.query_start
+    assert max_err(to_np(O)[qs:], ref["O"][qs:]) <= O_TOL
+    assert max_err(to_np(lse)[:, qs:], ref["lse"][:, qs:]) <= LSE_TOL
+    assert np.all(to_np(O)[:qs] == 0)            # rows outside the query block untouched
+    _no_device_error()
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_layer_fwd(name):
+    wl, lay, inp, ref = _case(name)
+    p = spava.Problem.from_workload(wl)
+    d = _dev(inp)
+    O, lse = spava.layer_fwd(p, d["Q"], d["K"], d["V"])
+    torch.cuda.synchronize()
+    _no_device_error()
+    On, ln = to_np(O), to_np(lse)
+    affected = {h: {kv: False for kv in range(lay.num_kv_heads)} for h in range(lay.V - 1)}
+    if wl.lp > 0:
+        # the layer's own selection, read back through the stage calls
+        _, scores = spava.score(p, d["Q"], d["K"])
+        idx = to_np(spava.select_topk(p, scores))
+        swaps, affected = compare_selection(lay, ref["scores"], ref["idx"], idx)
+    for r0, r1, h in [(0, lay.anchor_len, -1)] + \
+            [(lay.block_starts[h], lay.block_starts[h] + lay.block_lens[h], h) for h in range(lay.V)] + \
+            [(lay.query_start, lay.n, -1)]:
+        for g in range(wl.num_q_heads):
+            kv = g // lay.group
+            if h > 0 and host_affected(lay, affected, h, kv):
+                assert np.isfinite(On[r0:r1, g]).all()
+                continue
+            assert max_err(On[r0:r1, g], ref["O"][r0:r1, g]) <= O_TOL, (r0, g)
+            assert max_err(ln[g, r0:r1], ref["lse"][g, r0:r1]) <= LSE_TOL, (r0, g)
+
+
+def test_layer_is_deterministic_and_stream_ordered():
+    wl, lay, inp, ref = _case("frames_multi")
+    p = spava.Problem.from_workload(wl)
+    d = _dev(inp)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        O1, l1 = spava.layer_fwd(p, d["Q"], d["K"], d["V"], stream=s)
+        O2, l2 = spava.layer_fwd(p, d["Q"], d["K"], d["V"], stream=s)
+    s.synchronize()
+    assert torch.equal(O1, O2) and torch.equal(l1, l2)
+    _no_device_error()
+
+
+def test_bad_arguments_are_rejected_before_launch():
+    wl, lay, inp, ref = _case("tiny")
+    p = spava.Problem.from_workload(wl)
+    d = _dev(inp)
+    with pytest.raises(spava.SpavaError) as e:
+        spava.layer_fwd(p, d["Q"], d["K"], d["V"],
+                        workspace=torch.empty(16, dtype=torch.uint8, device="cuda"))
+    assert e.value.code == 3   # SPAVA_ERR_WORKSPACE
+    lib = spava.lib()
+    import ctypes
+    r = lib.spava_layer_fwd(p.ref, None, ctypes.c_void_p(d["K"].data_ptr()), ctypes.c_void_p(d["V"].data_ptr()),
+                            None, None, None, ctypes.c_size_t(0), None)
+    assert r == 1              # SPAVA_ERR_INVALID_ARG
+    mis = ctypes.c_void_p(d["Q"].data_ptr() + 2)
+    ws = torch.empty(spava.workspace_size(p), dtype=torch.uint8, device="cuda")
+    O = torch.empty_like(d["Q"])
+    lse = torch.empty(wl.num_q_heads, lay.n, device="cuda")
+    r = lib.spava_attn_fwd(p.ref, mis, ctypes.c_void_p(d["K"].data_ptr()), ctypes.c_void_p(d["V"].data_ptr()),
+                           ctypes.c_void_p(ws.data_ptr()), ctypes.c_void_p(ws.data_ptr()),
+                           ctypes.c_void_p(O.data_ptr()), ctypes.c_void_p(lse.data_ptr()),
+                           ctypes.c_void_p(ws.data_ptr()), ctypes.c_void_p(ws.data_ptr()), None)
+    assert r == 1              # misaligned Q
+    _no_device_error()
