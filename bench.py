@@ -1,0 +1,485 @@
+#!/usr/bin/env python
+"""Throughput of the approximate-attention prefill layer (Spava / APB-V) on
+B200, as prefill tokens/s per layer, with the attention kernel's achieved
+TFLOP/s against the measured bf16 tensor-core peak.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl reference]
+
+One step = one pass of the whole layer (query-block sum + score, top-lp,
+passing gather, attention, lse merge) over one synthetic input set, through
+the C ABI.  Timed on the device with CUDA events; inputs rotate over three
+resident sets so no step finds its inputs in L2.  With N > 1 (torchrun) every
+rank runs an independent replica of the layer on its own GPU (the layer does
+not shard: all virtual hosts live on one GPU) and the job value is the sum of
+tokens over the max over ranks of the elapsed time.
+
+--impl reference times the CPU fp64 oracle on the host cores instead (the
+reference arm: a bounded sample of the same workload per step).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "approx-attn prefill tokens/s per layer"
+DEFAULT_WORKLOAD = "qwen25vl3b_64f"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------ helpers
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def dist_init(world, backend):
+    import datetime
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def reduce_max(x: float, world: int, device=None) -> float:
+    """Max of a float over ranks (identity at world size 1)."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.index, self.proc, self.lines = self._smi_id(device), None, []
+
+    @staticmethod
+    def _smi_id(device) -> str:
+        """nvidia-smi id of a torch device (its UUID, so that a remapped
+        CUDA_VISIBLE_DEVICES still samples the right GPU)."""
+        try:
+            import torch
+            u = str(torch.cuda.get_device_properties(device).uuid)
+            return u if u.startswith("GPU-") else "GPU-" + u
+        except Exception:
+            return str(getattr(device, "index", 0) or 0)
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(self.index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def source_hash(path: str) -> str:
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def committed_traffic(workload: str):
+    """Per-launch DRAM bytes of the attention kernel from the committed ncu
+    summary, if it was taken on the current kernel source."""
+    p = os.path.join(ROOT, "profiles", "attn_kernel_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    src = os.path.join(ROOT, "sparse_approximate_attention_b200", "csrc", "attention.cuh")
+    e = d.get(workload)
+    if not e or e.get("source_sha256_16") != source_hash(src):
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------ oracle (CPU) arm
+def cpu_sample(wl, inp, n_tiles_per_host=1, nheads=2, seed=0):
+    """Time the oracle on a bounded sample of the workload: the whole
+    compression (scores + top-lp of every block), then one 128-row tile per
+    context block and the anchor, and the query rows, for a few heads.
+    Returns (tokens-equivalent processed, seconds, description, threads)."""
+    import numpy as np
+    import oracle
+    lay = oracle.make_layout(wl.num_hosts, wl.anchor_len, wl.block_lens, wl.query_len, wl.lp,
+                             wl.num_q_heads, wl.num_kv_heads, wl.head_dim)
+    heads = sorted(set(int(round(x)) for x in np.linspace(0, wl.num_q_heads - 1, nheads)))
+    rng = np.random.default_rng(seed)
+    t0 = time.perf_counter()
+    scores, idx = oracle.compress(lay, inp["Q"], inp["K"])
+    t_compress = time.perf_counter() - t0
+    rows = []
+    for h in range(lay.V):
+        s0, L = lay.block_starts[h], lay.block_lens[h]
+        for _ in range(n_tiles_per_host):
+            r0 = s0 + int(rng.integers(0, max(1, L - 128 + 1)))
+            rows += list(range(r0, min(s0 + L, r0 + 128)))
+    rows += list(range(min(128, lay.anchor_len)))
+    rows += list(range(lay.query_start, lay.n))
+    t1 = time.perf_counter()
+    oracle.rows_fwd(lay, inp["Q"], inp["K"], inp["V"], idx, rows, heads)
+    t_rows = time.perf_counter() - t1
+    frac = (len(rows) * len(heads)) / (lay.n * lay.num_q_heads)
+    tokens = lay.n * frac
+    secs = t_rows + t_compress * frac
+    desc = (f"oracle fp64 on {len(rows)} rows x {len(heads)} of {lay.num_q_heads} heads "
+            f"({n_tiles_per_host} random 128-row tile(s) per context block, first anchor tile, "
+            f"all query rows) "
+            f"= {frac:.4%} of the layer's row-heads; compression of all blocks "
+            f"({t_compress:.2f} s) charged pro rata")
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:  # pragma: no cover
+        threads = os.cpu_count()
+    return tokens, secs, desc, threads
+
+
+def run_reference(args, wl):
+    import torch  # noqa: F401  (generator)
+    from sparse_approximate_attention_b200 import workloads as W
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    inp = W.make_inputs(wl)
+    sz_n = wl.seq_len
+    for _ in range(args.warmup):
+        cpu_sample(wl, inp, seed=99)
+    tok, secs = 0.0, 0.0
+    desc, thr = "", 1
+    for k in range(args.steps):
+        t, s, desc, thr = cpu_sample(wl, inp, seed=k)
+        tok += t
+        secs += s
+    value = tok / secs
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * secs / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(wl, sz_n),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": thr, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(wl, n):
+    return {"workload": wl.name, "seq_len": n, "num_hosts": wl.num_hosts,
+            "virtual_hosts": 2 * wl.num_hosts, "anchor_len": wl.anchor_len,
+            "block_lens": sorted(set(wl.block_lens)) if len(set(wl.block_lens)) == 1 else wl.block_lens,
+            "query_len": wl.query_len, "lp": wl.lp, "q_heads": wl.num_q_heads,
+            "kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
+            "parallelism": "replicas (one independent layer per GPU)",
+            "l2": "3 rotating input sets, each larger than L2"}
+
+
+# ------------------------------------------------------------------ GPU arm
+def run_gpu(args, wl):
+    import torch
+    import sparse_approximate_attention_b200 as spava
+    from sparse_approximate_attention_b200 import workloads as W
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist_init(world, "nccl")
+    p = spava.Problem.from_workload(wl)
+    sz = p.sizes()
+    n = sz["seq_len"]
+    # three resident input sets (different seeds), each > L2
+    sets = []
+    host_inp = None
+    for i in range(3):
+        inp = W.make_inputs(wl, seed=wl.seed + 1000 * rank + i)
+        if i == 0:
+            host_inp = inp
+        sets.append({k: inp[k].to(dev) for k in ("Q", "K", "V")})
+    hq, hkv, d, V, lq, lp = wl.num_q_heads, wl.num_kv_heads, wl.head_dim, 2 * wl.num_hosts, wl.query_len, wl.lp
+    f32, bf = torch.float32, torch.bfloat16
+    O = torch.empty(n, hq, d, dtype=bf, device=dev)
+    lse = torch.empty(hq, n, dtype=f32, device=dev)
+    qsum = torch.empty(hkv, d, dtype=f32, device=dev)
+    scores = torch.empty(hkv, sz["score_cols"], dtype=f32, device=dev)
+    idx = torch.empty(V - 1, hkv, lp, dtype=torch.int32, device=dev)
+    Kp = torch.empty(max(1, sz["passing_rows"]), hkv, d, dtype=bf, device=dev)[: sz["passing_rows"]]
+    Vp = torch.empty_like(Kp)
+    O_part = torch.empty(V, lq, hq, d, dtype=f32, device=dev)
+    lse_part = torch.empty(V, hq, lq, dtype=f32, device=dev)
+    ws = torch.empty(sz["workspace_bytes"], dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    stages = ["score", "topk", "gather", "attn", "merge"]
+
+    def step(s, ev=None):
+        x = sets[s % 3]
+        if lp > 0:
+            spava.score(p, x["Q"], x["K"], qsum, scores, stream=stream)
+            if ev: ev[0].record(stream)
+            spava.select_topk(p, scores, idx, stream=stream)
+            if ev: ev[1].record(stream)
+            spava.gather_passing(p, x["K"], x["V"], idx, Kp, Vp, stream=stream)
+        elif ev:
+            ev[0].record(stream); ev[1].record(stream)
+        if ev: ev[2].record(stream)
+        spava.attn_fwd(p, x["Q"], x["K"], x["V"], Kp if lp else None, Vp if lp else None,
+                       O, lse, O_part, lse_part, stream=stream)
+        if ev: ev[3].record(stream)
+        spava.lse_merge(p, O_part, lse_part, O, lse, stream=stream)
+        if ev: ev[4].record(stream)
+
+    launches_per_step = (4 if lp > 0 else 0) + 2   # qsum, score, topk, gather | attn, merge
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    assert spava.device_error() == 0
+
+    # ---------------- timed region: K steps, per-stage events on the launch stream
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    t_begin = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev) as clk:
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        t_begin.record(stream)
+        for k in range(args.steps):
+            starts[k].record(stream)
+            step(k, ev[k])
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+    elapsed_ms = t_begin.elapsed_time(t_end)
+    elapsed_ms = reduce_max(elapsed_ms, world, dev)
+    err = spava.device_error()
+    assert err == 0, f"device error word {err}"
+    stage_ms = {s: 0.0 for s in stages}
+    for k in range(args.steps):
+        marks = [starts[k]] + ev[k]
+        for si, s in enumerate(stages):
+            stage_ms[s] += marks[si].elapsed_time(marks[si + 1])
+    stage_ms = {s: v / args.steps for s, v in stage_ms.items()}
+    ms_per_step = elapsed_ms / args.steps
+    value = world * n / (ms_per_step / 1000.0)
+
+    # ---------------- fused entry point, device-only (cross-check of the same work)
+    for i in range(3):
+        spava.layer_fwd(p, sets[i % 3]["Q"], sets[i % 3]["K"], sets[i % 3]["V"], O, lse, ws, stream=stream)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    a.record(stream)
+    for k in range(args.steps):
+        x = sets[k % 3]
+        spava.layer_fwd(p, x["Q"], x["K"], x["V"], O, lse, ws, stream=stream)
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    fused_ms = a.elapsed_time(b) / args.steps
+
+    if args.no_e2e:
+        e2e_ms, e2e_value, h2d, d2h = None, None, 0, 0
+    else:
+        e2e_ms, e2e_value, h2d, d2h = e2e_measure(p, host_inp, sets, O, lse, ws, stream, dev,
+                                                   world, n, args.steps)
+    if rank != 0:
+        return 0
+    return report(args, wl, sz, world, n, ms_per_step, value, stage_ms, stages, fused_ms,
+                  e2e_ms, e2e_value, h2d, d2h, launches_per_step, clk, host_inp)
+
+
+def e2e_measure(p, host_inp, sets, O, lse, ws, stream, dev, world, n, steps):
+    """The layer through the public call, with the H2D copy of the step's
+    inputs from pinned host memory and the D2H read of O and lse inside the
+    timed region."""
+    import torch
+    import sparse_approximate_attention_b200 as spava
+    bf, f32 = torch.bfloat16, torch.float32
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    hQ, hK, hV = (host_inp[k].pin_memory() for k in ("Q", "K", "V"))
+    hO = torch.empty(O.shape, dtype=bf).pin_memory()
+    hL = torch.empty(lse.shape, dtype=f32).pin_memory()
+    dQ, dK, dV = (torch.empty_like(sets[0][k]) for k in ("Q", "K", "V"))
+    h2d = sum(t.numel() * t.element_size() for t in (hQ, hK, hV))
+    d2h = hO.numel() * hO.element_size() + hL.numel() * hL.element_size()
+
+    def e2e_step():
+        dQ.copy_(hQ, non_blocking=True)
+        dK.copy_(hK, non_blocking=True)
+        dV.copy_(hV, non_blocking=True)
+        spava.layer_fwd(p, dQ, dK, dV, O, lse, ws, stream=stream)
+        hO.copy_(O, non_blocking=True)
+        hL.copy_(lse, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    a.record(stream)
+    e2e_steps = max(3, steps // 2)
+    for _ in range(e2e_steps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = reduce_max(a.elapsed_time(b) / e2e_steps, world, dev)
+    return e2e_ms, world * n / (e2e_ms / 1000.0), h2d, d2h
+
+
+def report(args, wl, sz, world, n, ms_per_step, value, stage_ms, stages, fused_ms, e2e_ms,
+           e2e_value, h2d, d2h, launches_per_step, clk, host_inp):
+    hq, hkv, d, V, lq, lp = (wl.num_q_heads, wl.num_kv_heads, wl.head_dim, 2 * wl.num_hosts,
+                             wl.query_len, wl.lp)
+    pk, src = peaks()
+    peak_tf = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    hbm = pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    flops = sz["attn_flops"]
+    attn_tf = flops / (stage_ms["attn"] / 1000.0) / 1e12
+    # algorithmic bytes of the HBM-bound stages
+    S, P = sz["score_cols"], sz["passing_rows"]
+    by = {
+        "score": hkv * S * d * 2 + hkv * S * 4 + lq * hq * d * 2,
+        "topk": hkv * S * 4 + (V - 1) * hkv * lp * 4,
+        "gather": 2 * 2 * P * hkv * d * 2 + (V - 1) * hkv * lp * 4,
+        "merge": V * lq * hq * (d + 1) * 4 + lq * hq * (d * 2 + 4),
+    }
+    stage_info = {}
+    for s in stages:
+        e = {"ms": round(stage_ms[s], 5)}
+        if s == "attn":
+            e.update(tflops=round(attn_tf, 1), frac_of_peak=round(attn_tf / peak_tf, 4))
+        elif stage_ms[s] > 0:
+            gbs = by[s] / (stage_ms[s] / 1000.0) / 1e9
+            e.update(algo_bytes=by[s], gbs=round(gbs, 1), frac_of_hbm=round(gbs / hbm, 4))
+        stage_info[s] = e
+    clocks = clk.summary()
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded long-video-shaped Q/K/V: rank-16 per-frame K/V + noise, "
+                "query block correlated with 2% of context keys)",
+        "config": config_of(wl, n),
+        "tflops_layer": round(flops / (ms_per_step / 1000.0) / 1e12, 1),
+        "roofline": {"bound": "tensor", "kernel": f"attn_kernel<{d}>", "achieved": round(attn_tf, 1),
+                     "peak": peak_tf, "unit": "TFLOP/s", "frac": round(attn_tf / peak_tf, 4),
+                     "traffic": committed_traffic(wl.name),
+                     "peak_source": f"bf16_tflops_sustained of {src} (kernel timed inside a "
+                                    f"back-to-back step loop)",
+                     "algorithmic_flops_per_launch": flops},
+        "stages": stage_info,
+        "fused_layer_ms": round(fused_ms, 4),
+        "e2e": None if e2e_ms is None else {
+            "value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3),
+            "api": "spava_layer_fwd with pinned-host H2D of Q,K,V and D2H of O,lse"},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        tok, secs, desc, thr = cpu_sample(wl, host_inp, n_tiles_per_host=2, nheads=4)
+        line["cpu_baseline"] = {"value": tok / secs, "unit": "tokens/s", "cores": thr,
+                                "kind": "oracle", "sample": desc, "seconds": round(secs, 2)}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="spava", choices=["spava", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    from sparse_approximate_attention_b200 import workloads as W
+    wl = W.workloads()[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, wl)
+    rc = run_gpu(args, wl)
+    rank, world, _ = dist_env()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return rc
+
+
+if __name__ == "__main__":
+    sys.exit(main())

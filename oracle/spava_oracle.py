@@ -131,19 +131,32 @@ def _f64(x) -> np.ndarray:
     return np.asarray(x, dtype=np.float64)
 
 
+def _take(T, rows, head) -> np.ndarray:
+    """T[rows, head, :] widened to float64 (index first, so only the rows
+    used are ever widened)."""
+    try:
+        import torch
+        if isinstance(T, torch.Tensor):
+            r = torch.as_tensor(np.asarray(rows, dtype=np.int64))
+            return T[r, head].to(torch.float64).numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.asarray(T[np.asarray(rows, dtype=np.int64), head], dtype=np.float64)
+
+
 # --------------------------------------------------------------------------
 # step 1: KV importance  ([SC] Fig. 5 caption "Q_qr K^T estimates KV
 # importance"; [PR] "What carries the argument"; reading R1)
 # --------------------------------------------------------------------------
 def importance_scores(lay: Layout, Q, K, h: int) -> np.ndarray:
     """fp64 scores [Hkv, L_h] of block h's keys against the query block."""
-    Qn, Kn = _f64(Q), _f64(K)
     qs, s0, L = lay.query_start, lay.block_starts[h], lay.block_lens[h]
     G, d = lay.group, lay.head_dim
     out = np.empty((lay.num_kv_heads, L))
+    qrows = np.arange(qs, qs + lay.query_len)
     for kv in range(lay.num_kv_heads):
-        q = Qn[qs:qs + lay.query_len, kv * G:(kv + 1) * G, :].reshape(-1, d)
-        k = Kn[s0:s0 + L, kv, :]
+        q = np.stack([_take(Q, qrows, g) for g in range(kv * G, (kv + 1) * G)], axis=1).reshape(-1, d)
+        k = _take(K, np.arange(s0, s0 + L), kv)
         logits = lay.scale * (q @ k.T)          # the Q_qr K^(h)T matrix
         out[kv] = logits.sum(axis=0)            # one importance per key
     return out
@@ -254,7 +267,6 @@ def context_rows(lay: Layout, Q, K, V, idx, h: int, rows: Sequence[int],
                  heads: Sequence[int]) -> Tuple[np.ndarray, np.ndarray]:
     """Rows (global positions inside B^(h), or inside B_a when h == -1) for
     the given query heads -> (o [len(rows), len(heads), d], lse [len(heads), len(rows)])."""
-    Qn, Kn, Vn = _f64(Q), _f64(K), _f64(V)
     rows = np.asarray(rows, dtype=np.int64)
     o = np.empty((len(rows), len(heads), lay.head_dim))
     lse = np.empty((len(heads), len(rows)))
@@ -271,7 +283,7 @@ def context_rows(lay: Layout, Q, K, V, idx, h: int, rows: Sequence[int],
         visible = np.zeros((len(rows), len(keys)), dtype=bool)
         visible[:, :len(fixed)] = True
         visible[:, len(fixed):] = local[None, :] <= rows[:, None]
-        oo, ll = attend(Qn[rows, g, :], Kn[keys, kv, :], Vn[keys, kv, :],
+        oo, ll = attend(_take(Q, rows, g), _take(K, keys, kv), _take(V, keys, kv),
                         lay.scale, visible)
         o[:, hi, :], lse[hi] = oo, ll
     return o, lse
@@ -280,7 +292,6 @@ def context_rows(lay: Layout, Q, K, V, idx, h: int, rows: Sequence[int],
 def query_partials(lay: Layout, Q, K, V, heads: Optional[Sequence[int]] = None):
     """Per-host partials of the query rows:
     o_part [V, lq, len(heads), d], lse_part [V, len(heads), lq]."""
-    Qn, Kn, Vn = _f64(Q), _f64(K), _f64(V)
     heads = list(range(lay.num_q_heads)) if heads is None else list(heads)
     rows = np.arange(lay.query_start, lay.n)
     o = np.empty((lay.V, len(rows), len(heads), lay.head_dim))
@@ -290,7 +301,7 @@ def query_partials(lay: Layout, Q, K, V, heads: Optional[Sequence[int]] = None):
             kv = g // lay.group
             keys = query_partial_positions(lay, h, lay.n - 1)
             visible = keys[None, :] <= rows[:, None]
-            oo, ll = attend(Qn[rows, g, :], Kn[keys, kv, :], Vn[keys, kv, :],
+            oo, ll = attend(_take(Q, rows, g), _take(K, keys, kv), _take(V, keys, kv),
                             lay.scale, visible)
             o[h, :, hi, :], lse[h, hi] = oo, ll
     return o, lse
@@ -348,7 +359,6 @@ def gather_passing(lay: Layout, K, V, idx) -> Tuple[np.ndarray, np.ndarray]:
     0..V-2 in host order): row (off_h + t, kv) holds key start_h + idx_h[kv][t]
     of KV head kv.  This is the single-GPU stand-in for the all-gather of
     passing blocks ([PR] "What carries the argument")."""
-    Kn, Vn = _f64(K), _f64(V)
     rows = sum(lay.lp_eff(h) for h in range(lay.V - 1))
     Kp = np.zeros((rows, lay.num_kv_heads, lay.head_dim))
     Vp = np.zeros_like(Kp)
@@ -357,8 +367,8 @@ def gather_passing(lay: Layout, K, V, idx) -> Tuple[np.ndarray, np.ndarray]:
         e = lay.lp_eff(h)
         for kv in range(lay.num_kv_heads):
             pos = lay.block_starts[h] + np.asarray(idx[h][kv], dtype=np.int64)
-            Kp[off:off + e, kv] = Kn[pos, kv]
-            Vp[off:off + e, kv] = Vn[pos, kv]
+            Kp[off:off + e, kv] = _take(K, pos, kv)
+            Vp[off:off + e, kv] = _take(V, pos, kv)
         off += e
     return Kp, Vp
 

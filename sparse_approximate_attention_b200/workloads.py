@@ -111,6 +111,12 @@ def workloads() -> Dict[str, Workload]:
         query_len=128, lp=8192, num_q_heads=16, num_kv_heads=2, head_dim=128,
         generator="frames", seed=1239,
         description="3B shape with lp = full block length (dense-exact)")
+    w["qwen25vl3b_h2"] = Workload(
+        "qwen25vl3b_h2", num_hosts=2, anchor_len=1024, block_lens=[8192] * 4,
+        query_len=128, lp=1024, num_q_heads=16, num_kv_heads=2, head_dim=128,
+        generator="frames", seed=1240,
+        description="half of the 3B-shaped layer (H=2/V=4, anchor 1024 + 4x8192 + "
+        "query 128, lp=1024): the profiling case, inputs still larger than L2")
     blens = _unequal_blocks(1239, 8, 65536, 4096, 12288)
     w["exact_dense_3b_unequal"] = Workload(
         "exact_dense_3b_unequal", num_hosts=4, anchor_len=1024, block_lens=blens,
