@@ -150,6 +150,28 @@ spava_status_t spava_layer_fwd(const spava_problem_t* prob, const void* Q,
                                float* lse, void* workspace, size_t ws_bytes,
                                spava_stream_t stream);
 
+/* The whole layer, like spava_layer_fwd, for callers that cannot allocate
+ * device memory: code that only receives input and output pointers from a
+ * host framework which owns the device allocator (a plugin or operator
+ * interface), or whose memory budget leaves no room to reserve a separate
+ * workspace, and so cannot hand this library a workspace.  The pages describe
+ * no such entry; it has no counterpart in the paper.
+ *
+ * The intermediates live instead in one fixed array of 64 MiB inside this
+ * library: every GPU that loads the library holds it until the process
+ * exits.  A problem whose workspace (spava_workspace_size) exceeds 64 MiB is
+ * rejected with SPAVA_ERR_WORKSPACE before anything is launched.  The call
+ * allocates no device memory.  Its first call on a device looks up the
+ * array's device address on that device (cudaGetSymbolAddress); make that
+ * first call before any stream capture.  All calls on a device share the
+ * array and it keeps the last call's contents (nothing in it needs to start
+ * at zero: each call writes every byte it reads).  Calls whose work overlaps
+ * on the GPU (other streams, other host threads) race on the array and give
+ * wrong results: serialise them. */
+spava_status_t spava_layer_fwd_noalloc(const spava_problem_t* prob, const void* Q,
+                                       const void* K, const void* V, void* O,
+                                       float* lse, spava_stream_t stream);
+
 /* Device-side error word of the current device (0 = none); synchronizes the
  * device, then clears the word.  Bit 0: a bounded wait in the attention
  * kernel gave up. */

@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstring>
 #include <memory>
+#include <mutex>
 #include <vector>
 
 #include "../../include/spava.h"
@@ -329,3 +330,64 @@ const char* spava_status_string(spava_status_t status) {
 }
 
 }  // extern "C"
+
+// ======================================================= no-allocation entry
+// A copy of the layer's sequencing whose intermediates live in a fixed
+// device array of this library instead of a caller-provided workspace.
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(64) << 20;   // 64 MiB per device
+__device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
+
+constexpr int kMaxScratchDevices = 64;
+std::mutex g_static_scratch_mu;
+void* g_static_scratch_addr[kMaxScratchDevices] = {};
+
+// Device address of g_static_scratch on the current device.  The first call
+// on a device looks it up (cudaGetSymbolAddress, with that device current)
+// and keeps it; later calls reuse it.
+spava_status_t static_scratch_address(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SPAVA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxScratchDevices) return SPAVA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_static_scratch_mu);
+  if (!g_static_scratch_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return SPAVA_ERR_CUDA;
+    g_static_scratch_addr[dev] = p;
+  }
+  *out = g_static_scratch_addr[dev];
+  return SPAVA_OK;
+}
+
+}  // namespace
+
+extern "C" spava_status_t spava_layer_fwd_noalloc(const spava_problem_t* prob, const void* Q,
+                                                  const void* K, const void* V, void* O, float* lse,
+                                                  spava_stream_t stream) {
+  Plan P;
+  spava_status_t s = make_plan(prob, &P);
+  if (s != SPAVA_OK) return s;
+  if (P.ws_total > kStaticScratchBytes) return SPAVA_ERR_WORKSPACE;   // problem too large for it
+  if (!Q || !K || !V || !O || !lse) return SPAVA_ERR_INVALID_ARG;
+  void* base = nullptr;
+  if ((s = static_scratch_address(&base)) != SPAVA_OK) return s;
+  // Every byte the steps below read from the scratch is written earlier in
+  // the same call, so nothing has to be cleared between calls.
+  auto* ws = static_cast<uint8_t*>(base);
+  float* qsum = reinterpret_cast<float*>(ws + P.ws_qsum);
+  float* scores = reinterpret_cast<float*>(ws + P.ws_scores);
+  int32_t* idx = reinterpret_cast<int32_t*>(ws + P.ws_idx);
+  void* Kp = ws + P.ws_kp;
+  void* Vp = ws + P.ws_vp;
+  float* O_part = reinterpret_cast<float*>(ws + P.ws_opart);
+  float* lse_part = reinterpret_cast<float*>(ws + P.ws_lsepart);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (P.lp > 0) {
+    if ((s = run_score(P, Q, K, qsum, scores, st)) != SPAVA_OK) return s;
+    if ((s = run_topk(P, scores, idx, st)) != SPAVA_OK) return s;
+    if ((s = run_gather(P, K, V, idx, Kp, Vp, st)) != SPAVA_OK) return s;
+  }
+  if ((s = run_attn(P, Q, K, V, Kp, Vp, O, lse, O_part, lse_part, st)) != SPAVA_OK) return s;
+  return run_merge(P, O_part, lse_part, O, lse, st);
+}

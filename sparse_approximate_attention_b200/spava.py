@@ -238,3 +238,20 @@ def device_error() -> int:
     v = ctypes.c_uint32()
     _check("spava_device_error", lib().spava_device_error(ctypes.byref(v)))
     return v.value
+
+
+def layer_fwd_noalloc(p: Problem, Q, K, V, O, lse, stream=None):
+    """The whole layer without a workspace, for callers that cannot allocate
+    device memory: its intermediates live in a fixed 64 MiB array inside the
+    library (problems whose workspace is larger are rejected).  O and lse are
+    caller-provided.  Calls that overlap on the GPU race on that array."""
+    sz, sh = _shapes(p)
+    for t, nm in ((Q, "Q"), (K, "K"), (V, "V"), (O, "O")):
+        _need(t, torch.bfloat16, sh[nm], nm)
+    _need(lse, torch.float32, sh["lse"], "lse")
+    f = lib().spava_layer_fwd_noalloc
+    f.argtypes = [_PP, _VP, _VP, _VP, _VP, _VP, _VP]
+    f.restype = ctypes.c_int
+    _check("spava_layer_fwd_noalloc", f(p.ref, _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(lse),
+                                        _stream(stream)))
+    return O, lse
