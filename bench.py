@@ -459,7 +459,7 @@ def report(args, wl, sz, world, n, ms_per_step, value, stage_ms, stages, fused_m
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="spava", choices=["spava", "reference"])

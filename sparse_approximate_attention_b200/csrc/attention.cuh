@@ -1,8 +1,9 @@
 // Variable-segment causal attention on tcgen05 / TMEM with TMA-fed tiles.
 //
-// One CTA computes one 128-row tile of one query head.  Its keys are a list
-// of up to three segments (rows of K/V or of the passing buffer Kp/Vp), which
-// covers every row kind of the layer in a single launch:
+// One CTA computes two consecutive 128-row tiles (Q0, Q1) of one query head
+// that share one key list.  The key list is up to three segments (rows of
+// K/V or of the passing buffer Kp/Vp), which covers every row kind of the
+// layer in a single launch:
 //   anchor rows            : causal over B_a
 //   context rows of host h : B_a, Kp rows of hosts < h, causal B^(h)
 //                            ("APB-V ..." pith.science review, minor comment
@@ -14,14 +15,21 @@
 // The launch's CTAs are ordered longest key list first (Fig. 4, attention
 // load balancing).
 //
-// Warp roles (192 threads):
-//   warp 0     TMA producer: Q once, then K and V tiles into a ring of stages
-//   warp 1     TMEM owner and MMA issuer: S = Q K^T into one of two TMEM
-//              buffers, then O += P V with P read from TMEM
-//   warps 2-5  softmax: one thread per query row, online softmax in the
-//              exp2 domain with a lazy rescale of O (only when the running
-//              max grows by more than 2^8), P written back to TMEM as bf16
-// TMEM columns: O [0, D), S/P buffer b at [128 + 128 b, 256 + 128 b).
+// Warp roles (384 threads, three warpgroups; the first gives registers to the
+// other two with setmaxnreg):
+//   warp 0     TMA producer: Q0 and Q1 once, then K and V tiles into separate
+//              rings (K runs one tile ahead of V, the order the MMAs use them)
+//   warp 1     TMEM owner and single-thread MMA issuer.  Per key tile j:
+//              S0 = Q0 K_j^T, O1 += P1 V_{j-1}, S1 = Q1 K_j^T, O0 += P0 V_j,
+//              so the tensor pipe works on one tile while the other tile's
+//              softmax runs
+//   warps 2-3  idle (they complete warpgroup 0)
+//   warps 4-7  softmax of Q0, warps 8-11 softmax of Q1: one thread per row,
+//              online softmax in the exp2 domain (3/8 of the exponentials on
+//              the FMA pipe, packed f32x2 arithmetic), lazy rescale of O (only
+//              when the row max grows by more than 2^8), P written back to
+//              TMEM as bf16 over S
+// TMEM columns: O0 [0, D), O1 [128, 128 + D), S0/P0 [256, 384), S1/P1 [384, 512).
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -41,7 +49,7 @@ struct AttnParams {
   float scale_log2;
   int32_t nregions, nitems;
   Region regions[kMaxRegions];
-  uint32_t items[kMaxItems];
+  uint32_t items[kMaxItems];   // (region << 20) | pair of 128-row tiles
 };
 static_assert(sizeof(AttnParams) <= 32764, "kernel parameter block too large");
 
@@ -50,17 +58,19 @@ struct AttnCfg {
   static constexpr int kSlabs = D / 64;                  // 128-byte-wide column slabs
   static constexpr int kSlabBytes = 128 * 128;           // 128 rows x 128 B
   static constexpr int kTileBytes = kSlabs * kSlabBytes;
-  static constexpr int kKStages = (D == 128) ? 3 : 4;    // K ring (released after S = Q K^T)
-  static constexpr int kVStages = (D == 128) ? 2 : 4;    // V ring (released after O += P V)
-  static constexpr int kOffQ = 0;
-  static constexpr int kOffK = kTileBytes;
+  static constexpr int kKStages = (D == 128) ? 3 : 4;    // K ring (released after both S MMAs)
+  static constexpr int kVStages = (D == 128) ? 2 : 4;    // V ring (released after both PV MMAs)
+  static constexpr int kOffQ = 0;                        // Q0, Q1
+  static constexpr int kOffK = 2 * kTileBytes;
   static constexpr int kOffV = kOffK + kKStages * kTileBytes;
   static constexpr int kOffBar = kOffV + kVStages * kTileBytes;
-  // barriers: Q, Kfull[KS], Kempty[KS], Vfull[VS], Vempty[VS], Sfull[2], Pfull[2], Odone, Fin
-  static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 2 + 2 + 1 + 1;
+  // barriers: Q, Kfull[KS], Kempty[KS], Vfull[VS], Vempty[VS], Sfull[2], Pfull[2], Odone[2], Fin
+  static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 1;
   static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;   // + slack for 1 KB alignment
-  static constexpr int kThreads = 192;
+  static constexpr int kThreads = 384;
+  static constexpr uint32_t kRegsLow = 56;     // warpgroup 0: producer, MMA issuer
+  static constexpr uint32_t kRegsHigh = 224;   // warpgroups 1, 2: softmax
   static constexpr uint32_t kTmemCols = 512;
 };
 static_assert(AttnCfg<128>::kSmemBytes <= 232448, "shared memory budget");
@@ -82,10 +92,10 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1)
   auto BAR_KE = [&](int s) { return bar0 + 8u * (1 + KS + s); };
   auto BAR_VF = [&](int s) { return bar0 + 8u * (1 + 2 * KS + s); };
   auto BAR_VE = [&](int s) { return bar0 + 8u * (1 + 2 * KS + VS + s); };
-  auto BAR_SF = [&](int b) { return bar0 + 8u * (1 + 2 * KS + 2 * VS + b); };
-  auto BAR_PF = [&](int b) { return bar0 + 8u * (3 + 2 * KS + 2 * VS + b); };
-  const uint32_t BAR_OD = bar0 + 8u * (5 + 2 * KS + 2 * VS);
-  const uint32_t BAR_FIN = bar0 + 8u * (6 + 2 * KS + 2 * VS);
+  auto BAR_SF = [&](int t) { return bar0 + 8u * (1 + 2 * KS + 2 * VS + t); };
+  auto BAR_PF = [&](int t) { return bar0 + 8u * (3 + 2 * KS + 2 * VS + t); };
+  auto BAR_OD = [&](int t) { return bar0 + 8u * (5 + 2 * KS + 2 * VS + t); };
+  const uint32_t BAR_FIN = bar0 + 8u * (7 + 2 * KS + 2 * VS);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
@@ -93,38 +103,46 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1)
   const uint32_t item = p.items[blockIdx.x / p.Hq];
   const int head = blockIdx.x % p.Hq;
   const Region& R = p.regions[item >> 20];
-  const int tile = static_cast<int>(item & 0xFFFFFu);
+  const int pair = static_cast<int>(item & 0xFFFFFu);
   const int kv = head / p.G;
-  const int row0 = R.row_start + tile * kBM;
-  const int rows_valid = min(kBM, R.nrows - tile * kBM);
-  const int r_last = row0 + rows_valid - 1;
+  const int row0 = R.row_start + pair * 2 * kBM;               // first row of Q0
+  const int rv0 = min(kBM, R.nrows - pair * 2 * kBM);          // valid rows of Q0 (>= 1)
+  const int rv1 = min(kBM, R.nrows - (pair * 2 + 1) * kBM);    // valid rows of Q1 (<= 0: none)
+  const bool has1 = rv1 > 0;
   const int nseg = R.nseg;
-  int nt[kMaxSegs];
-  int ntiles = 0;
+  // Key tiles per segment.  Q0's key tiles are a prefix of Q1's: only the
+  // trailing causal segment can reach further for Q1's later rows.
+  int ntks[kMaxSegs];
+  int nt0 = 0, ntk = 0;
 #pragma unroll
   for (int s = 0; s < kMaxSegs; ++s) {
-    int vis = 0;
+    int v0 = 0, v1 = 0;
     if (s < nseg) {
       const Seg& sg = R.seg[s];
-      vis = sg.causal ? max(0, min(sg.len, r_last - sg.start + 1)) : sg.len;
+      const int rl0 = row0 + rv0 - 1;
+      const int rl1 = has1 ? row0 + kBM + rv1 - 1 : rl0;
+      v0 = sg.causal ? max(0, min(sg.len, rl0 - sg.start + 1)) : sg.len;
+      v1 = sg.causal ? max(0, min(sg.len, rl1 - sg.start + 1)) : sg.len;
     }
-    nt[s] = (vis + kBN - 1) / kBN;
-    ntiles += nt[s];
+    nt0 += (v0 + kBN - 1) / kBN;
+    ntks[s] = (v1 + kBN - 1) / kBN;
+    ntk += ntks[s];
   }
-  // Walks the key tiles in order: segment s, tile kt within it.
+  const int nt1 = has1 ? ntk : 0;      // key tiles of Q1 (all loaded tiles)
+  // Walks the loaded key tiles in order: segment s, tile kt within it.
   struct TileIter {
     int s, kt;
   };
   auto iter_begin = [&]() {
     TileIter it{0, 0};
-    while (it.s < nseg && nt[it.s] == 0) ++it.s;
+    while (it.s < nseg && ntks[it.s] == 0) ++it.s;
     return it;
   };
   auto iter_next = [&](TileIter& it) {
-    if (++it.kt == nt[it.s]) {
+    if (++it.kt == ntks[it.s]) {
       it.kt = 0;
       ++it.s;
-      while (it.s < nseg && nt[it.s] == 0) ++it.s;
+      while (it.s < nseg && ntks[it.s] == 0) ++it.s;
     }
   };
 
@@ -138,11 +156,11 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1)
       mbar_init(BAR_VF(s), 1);
       mbar_init(BAR_VE(s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(BAR_SF(b), 1);
-      mbar_init(BAR_PF(b), 128);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(BAR_SF(t), 1);
+      mbar_init(BAR_PF(t), 128);
+      mbar_init(BAR_OD(t), 1);
     }
-    mbar_init(BAR_OD, 1);
     mbar_init(BAR_FIN, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -156,21 +174,23 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  if (warp < 4) setmaxnreg_dec<C::kRegsLow>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    // K runs one tile ahead of V, matching the order the MMA consumes them
-    // (S_j = Q K_j^T is issued before O += P_{j-1} V_{j-1}).
     if (lane == 0) {
       tma_prefetch_desc(&p.tm_q);
       tma_prefetch_desc(&p.tm_k);
       tma_prefetch_desc(&p.tm_v);
-      mbar_arrive_expect_tx(BAR_Q, C::kTileBytes);
-      for (int sl = 0; sl < C::kSlabs; ++sl)
-        tma_load_3d(sQ + sl * C::kSlabBytes, &p.tm_q, BAR_Q, sl * 64, head, row0);
+      const int nq = has1 ? 2 : 1;
+      mbar_arrive_expect_tx(BAR_Q, nq * C::kTileBytes);
+      for (int t = 0; t < nq; ++t)
+        for (int sl = 0; sl < C::kSlabs; ++sl)
+          tma_load_3d(sQ + t * C::kTileBytes + sl * C::kSlabBytes, &p.tm_q, BAR_Q, sl * 64, head,
+                      row0 + t * kBM);
       int k_issued = 0, v_issued = 0;
       TileIter ik = iter_begin(), iv = iter_begin();
-      for (int j = 0; j <= ntiles; ++j) {
-        if (j < ntiles) {
+      for (int j = 0; j <= ntk; ++j) {
+        if (j < ntk) {
           const int st = j % KS;
           if (j >= KS && !mbar_wait(BAR_KE(st), ((j / KS) - 1) & 1, abort_flag)) break;
           const Seg& sg = R.seg[ik.s];
@@ -206,114 +226,156 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t kIdescQK = idesc_bf16_f32(128, kBN, false, false);
       constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, false, true);
-      const uint32_t tO = tmem;
-      auto issue_pv = [&](int i) -> bool {
-        const int st = i % VS, b = i & 1;
-        if (!mbar_wait(BAR_PF(b), (i >> 1) & 1, abort_flag)) return false;
-        if (!mbar_wait(BAR_VF(st), (i / VS) & 1, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t tP = tmem + 128u + 128u * b;
-#pragma unroll
-        for (int k = 0; k < kBN / 16; ++k) {
-          const uint64_t bdesc = sw128_desc(sV + st * C::kTileBytes + k * 2048, C::kSlabBytes, 1024);
-          mma_ts(tO, tP + k * 8, bdesc, kIdescPV, (i > 0 || k > 0) ? 1u : 0u);
-        }
-        mma_commit(BAR_OD);
-        mma_commit(BAR_VE(st));
-        return true;
-      };
-      bool ok = mbar_wait(BAR_Q, 0, abort_flag);
-      for (int j = 0; ok && j < ntiles; ++j) {
-        const int st = j % KS, b = j & 1;
-        ok = mbar_wait(BAR_KF(st), (j / KS) & 1, abort_flag);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t tS = tmem + 128u + 128u * b;
+      // Descriptor high words are constant (SBO 1024 B, version 1, 128-B
+      // swizzle); the low word is (address >> 4) | (LBO >> 4) << 16, so
+      // stepping through a tile only adds to the low word.
+      constexpr uint32_t kDescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
+      auto desc = [](uint32_t lo) -> uint64_t { return (static_cast<uint64_t>(kDescHi) << 32) | lo; };
+      const uint32_t q_lo = (sQ >> 4) | (1u << 16);
+      const uint32_t k_lo = (sK >> 4) | (1u << 16);
+      const uint32_t v_lo = (sV >> 4) | ((static_cast<uint32_t>(C::kSlabBytes) >> 4) << 16);
+      // S_t = Q_t K_j^T into TMEM buffer t
+      auto issue_s = [&](int t, int j) {
+        const uint32_t tS = tmem + 256u + 128u * t;
+        const uint32_t qa = q_lo + ((t * C::kTileBytes) >> 4);
+        const uint32_t kb = k_lo + (((j % KS) * C::kTileBytes) >> 4);
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
-          const int sl = k >> 2, off = (k & 3) * 32;
-          const uint64_t adesc = sw128_desc(sQ + sl * C::kSlabBytes + off, 16, 1024);
-          const uint64_t bdesc = sw128_desc(sK + st * C::kTileBytes + sl * C::kSlabBytes + off, 16, 1024);
-          mma_ss(tS, adesc, bdesc, kIdescQK, k > 0 ? 1u : 0u);
+          const uint32_t off = ((k >> 2) * C::kSlabBytes + (k & 3) * 32) >> 4;
+          mma_ss(tS, desc(qa + off), desc(kb + off), kIdescQK, k > 0 ? 1u : 0u);
         }
-        mma_commit(BAR_SF(b));
-        mma_commit(BAR_KE(st));
-        if (j > 0) ok = issue_pv(j - 1);
+        mma_commit(BAR_SF(t));
+      };
+      // O_t += P_t V_j once P_t (softmax of tile t) and V_j are ready
+      // O_t += P_t V_j once P_t (softmax of tile t) is ready; V_j's arrival
+      // is awaited by the caller beforehand, off the P-ready path.
+      auto issue_pv = [&](int t, int j, bool release_v) -> bool {
+        if (!mbar_wait(BAR_PF(t), j & 1, abort_flag)) return false;
+        tc_fence_after();
+        const int st = j % VS;
+        const uint32_t tP = tmem + 256u + 128u * t;
+        const uint32_t tO = tmem + 128u * t;
+        const uint32_t vb = v_lo + ((st * C::kTileBytes) >> 4);
+#pragma unroll
+        for (int k = 0; k < kBN / 16; ++k)
+          mma_ts(tO, tP + k * 8, desc(vb + ((k * 2048) >> 4)), kIdescPV, (j > 0 || k > 0) ? 1u : 0u);
+        mma_commit(BAR_OD(t));
+        if (release_v) mma_commit(BAR_VE(st));
+        return true;
+      };
+      auto wait_v = [&](int j) { return mbar_wait(BAR_VF(j % VS), (j / VS) & 1, abort_flag); };
+      bool ok = mbar_wait(BAR_Q, 0, abort_flag);
+      for (int j = 0; ok && j < ntk; ++j) {
+        ok = mbar_wait(BAR_KF(j % KS), (j / KS) & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        if (j < nt0) issue_s(0, j);
+        if (j >= 1 && j - 1 < nt1) {
+          ok = issue_pv(1, j - 1, true);   // V_{j-1} arrived before O0 += P0 V_{j-1}
+          if (!ok) break;
+        }
+        if (j < nt1) issue_s(1, j);
+        mma_commit(BAR_KE(j % KS));
+        ok = wait_v(j);                    // V_j is needed by O0 (now) or O1 (next)
+        if (!ok) break;
+        if (j < nt0) {
+          ok = issue_pv(0, j, j >= nt1);   // V_j is Q0's alone when Q1 does not read it
+          if (!ok) break;
+        }
       }
-      if (ok && ntiles > 0) issue_pv(ntiles - 1);
+      if (ok && nt1 > 0) issue_pv(1, nt1 - 1, true);
       mma_commit(BAR_FIN);   // every MMA issued above has finished once this lands
       mbar_wait_drain(BAR_FIN, 0);
     }
-  } else {
+  } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax
+    setmaxnreg_inc<C::kRegsHigh>();
+    const int qt = warp >= 8 ? 1 : 0;       // which Q tile this warpgroup owns
+    const int nt = qt ? nt1 : nt0;
     const int q = warp & 3;                 // TMEM lane quarter of this warp
     const int rit = q * 32 + lane;          // row in tile
-    const int row = row0 + rit;
-    const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    const int row = row0 + qt * kBM + rit;
+    const int rows_valid = qt ? rv1 : rv0;
+    const uint32_t tq = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    const uint32_t tS = tq + 256u + 128u * qt;
+    const uint32_t tO = tq + 128u * qt;
     const float sl2 = p.scale_log2;
     float m = -INFINITY;   // running max of the scaled logits, log2 units
     float l = 0.f;
     bool ok = true;
-    int s = 0, kt = 0;
-    while (s < nseg && nt[s] == 0) ++s;
-    for (int j = 0; j < ntiles; ++j) {
-      const int b = j & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(BAR_SF(b), (j >> 1) & 1, abort_flag));
+    TileIter it = iter_begin();
+    for (int j = 0; j < nt; ++j) {
+      ok = __all_sync(0xffffffffu, mbar_wait(BAR_SF(qt), j & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      float x[kBN];
+      float2 x[kBN / 2];
 #pragma unroll
       for (int c = 0; c < kBN / 32; ++c) {
         uint32_t r[32];
-        tmem_ld32(taddr + 128u + 128u * b + c * 32, r);
+        tmem_ld32(tS + c * 32, r);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(r[e]);
+        for (int e = 0; e < 16; ++e)
+          x[c * 16 + e] = make_float2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]));
       }
       tmem_wait_ld();
-      const Seg& sg = R.seg[s];
+      const Seg& sg = R.seg[it.s];
       int lim = sg.len;
       if (sg.causal) lim = min(lim, row - sg.start + 1);
-      const int nvalid = lim - kt * kBN;
+      const int nvalid = lim - it.kt * kBN;
       if (nvalid < kBN) {
 #pragma unroll
-        for (int c = 0; c < kBN; ++c)
-          if (c >= nvalid) x[c] = -INFINITY;
+        for (int i = 0; i < kBN / 2; ++i) {
+          if (2 * i >= nvalid) x[i].x = -INFINITY;
+          if (2 * i + 1 >= nvalid) x[i].y = -INFINITY;
+        }
       }
-      float mx = x[0];
+      float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int c = 1; c < kBN; ++c) mx = fmaxf(mx, x[c]);
-      mx *= sl2;
+      for (int i = 0; i < kBN / 2; i += 4) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) mq[u] = fmax3(mq[u], x[i + u].x, x[i + u].y);
+      }
+      const float mx = fmax3(mq[0], mq[1], fmaxf(mq[2], mq[3])) * sl2;
       const bool grow = mx > m + 8.0f;
       const float m_new = grow ? mx : m;
       const float alpha = grow ? ex2_approx(m - m_new) : 1.0f;
-      const float neg = -m_new;
+      const float2 sl22 = make_float2(sl2, sl2);
+      const float2 neg2 = make_float2(-m_new, -m_new);
       uint32_t pk[kBN / 2];
-      float sum = 0.f;
+      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                       make_float2(0.f, 0.f)};
 #pragma unroll
-      for (int c = 0; c < kBN; c += 2) {
-        const float p0 = ex2_approx(fmaf(x[c], sl2, neg));
-        const float p1 = ex2_approx(fmaf(x[c + 1], sl2, neg));
-        sum += p0 + p1;
-        pk[c / 2] = pack_bf16x2(p0, p1);
+      for (int i = 0; i < kBN / 2; ++i) {
+        const float2 y = __ffma2_rn(x[i], sl22, neg2);
+        float2 pe;
+        if ((i & 7) < 3) {   // three pairs in eight on the FMA pipe, the rest on MUFU
+          pe = exp2_poly2(y);
+        } else {
+          pe = make_float2(ex2_approx(y.x), ex2_approx(y.y));
+        }
+        acc[i & 3] = __fadd2_rn(acc[i & 3], pe);
+        pk[i] = pack_bf16x2(pe.x, pe.y);
       }
-      l = l * alpha + sum;
+      const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
+      const float2 a4 = __fadd2_rn(a01, a23);
+      l = l * alpha + (a4.x + a4.y);
       m = m_new;
       if (j > 0) {
-        // O += P_{j-1} V_{j-1} must be complete before O is rescaled and
-        // before P_j may be consumed; waiting every tile keeps the barrier
-        // within one phase of this waiter.
-        ok = __all_sync(0xffffffffu, mbar_wait(BAR_OD, (j - 1) & 1, abort_flag));
+        // O_t += P V of the previous tile must be complete before O_t is
+        // rescaled and before P overwrites S; waiting every tile keeps the
+        // barrier within one phase of this waiter.
+        ok = __all_sync(0xffffffffu, mbar_wait(BAR_OD(qt), (j - 1) & 1, abort_flag));
         if (!ok) break;
         tc_fence_after();
         if (__any_sync(0xffffffffu, grow)) {
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t r[32];
-            tmem_ld32(taddr + c * 32, r);
+            tmem_ld32(tO + c * 32, r);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-            tmem_st32(taddr + c * 32, r);
+            tmem_st32(tO + c * 32, r);
           }
         }
       }
@@ -324,22 +386,18 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1)
           r0[e] = pk[e];
           r1[e] = pk[32 + e];
         }
-        tmem_st32(taddr + 128u + 128u * b, r0);
-        tmem_st32(taddr + 128u + 128u * b + 32, r1);
+        tmem_st32(tS, r0);
+        tmem_st32(tS + 32, r1);
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(BAR_PF(b));
-      if (++kt == nt[s]) {
-        kt = 0;
-        ++s;
-        while (s < nseg && nt[s] == 0) ++s;
-      }
+      mbar_arrive(BAR_PF(qt));
+      iter_next(it);
     }
-    if (ok && ntiles > 0) {
-      ok = __all_sync(0xffffffffu, mbar_wait(BAR_OD, (ntiles - 1) & 1, abort_flag));
+    if (ok && nt > 0) {
+      ok = __all_sync(0xffffffffu, mbar_wait(BAR_OD(qt), (nt - 1) & 1, abort_flag));
     }
-    if (ok) {
+    if (ok && nt > 0) {
       tc_fence_after();
       const bool valid = rit < rows_valid;
       const float inv_l = 1.0f / l;
@@ -349,7 +407,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1)
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t r[32];
-          tmem_ld32(taddr + c * 32, r);
+          tmem_ld32(tO + c * 32, r);
           tmem_wait_ld();
           if (valid) {
 #pragma unroll
@@ -370,7 +428,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1)
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t r[32];
-          tmem_ld32(taddr + c * 32, r);
+          tmem_ld32(tO + c * 32, r);
           tmem_wait_ld();
           if (valid) {
 #pragma unroll

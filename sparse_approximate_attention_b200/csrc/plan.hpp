@@ -184,22 +184,27 @@ inline spava_status_t make_plan(const spava_problem_t* p, Plan* pl) {
   return SPAVA_OK;
 }
 
-// Cost-ordered work items: (region << 20) | tile, longest key list first.
+// Cost-ordered work items: (region << 20) | pair, one CTA per pair of
+// consecutive 128-row tiles of a region, longest key list first.  A pair
+// without its second tile costs about two thirds of a full one per key tile
+// (the softmax of one tile is then exposed).
 inline spava_status_t make_items(const Plan& P, std::vector<uint32_t>* items) {
   struct It {
     int64_t cost;
     uint32_t code;
   };
   std::vector<It> v;
-  v.reserve(static_cast<size_t>(P.tiles));
+  v.reserve(static_cast<size_t>(P.tiles / 2 + P.nregions));
   for (int r = 0; r < P.nregions; ++r) {
     const Region& R = P.regions[r];
-    int nt = (R.nrows + kBM - 1) / kBM;
-    for (int t = nt - 1; t >= 0; --t) {
-      int64_t r_last = R.row_start + std::min(R.nrows, (t + 1) * kBM) - 1;
+    const int nt = (R.nrows + kBM - 1) / kBM;
+    const int np = (nt + 1) / 2;
+    for (int q = np - 1; q >= 0; --q) {
+      const bool two = 2 * q + 1 < nt;
+      const int64_t r_last = R.row_start + std::min(R.nrows, (2 * q + (two ? 2 : 1)) * kBM) - 1;
       int64_t ktiles = 0;
       for (int s = 0; s < R.nseg; ++s) ktiles += (seg_visible_len(R.seg[s], r_last) + kBN - 1) / kBN;
-      v.push_back(It{ktiles, (static_cast<uint32_t>(r) << 20) | static_cast<uint32_t>(t)});
+      v.push_back(It{ktiles * (two ? 3 : 2), (static_cast<uint32_t>(r) << 20) | static_cast<uint32_t>(q)});
     }
   }
   if (v.size() > static_cast<size_t>(kMaxItems)) return SPAVA_ERR_UNSUPPORTED;

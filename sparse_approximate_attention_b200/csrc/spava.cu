@@ -147,6 +147,13 @@ spava_status_t launch_attn(const AttnParams& prm, int grid, cudaStream_t st) {
   if (cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
       cudaSuccess)
     return SPAVA_ERR_CUDA;
+  // The kernel moves registers from warpgroup 0 to the softmax warpgroups
+  // (setmaxnreg); refuse to launch unless the launch allocation covers that
+  // split, since an uncovered increase would never be granted.
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, attn_kernel<D>) != cudaSuccess) return SPAVA_ERR_CUDA;
+  if (static_cast<long>(fa.numRegs) * C::kThreads < 128L * C::kRegsLow + 256L * C::kRegsHigh)
+    return SPAVA_ERR_UNSUPPORTED;
   attn_kernel<D><<<grid, C::kThreads, C::kSmemBytes, st>>>(prm);
   return last_launch();
 }
