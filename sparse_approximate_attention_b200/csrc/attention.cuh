@@ -64,8 +64,9 @@ struct AttnCfg {
   static constexpr int kOffK = 2 * kTileBytes;
   static constexpr int kOffV = kOffK + kKStages * kTileBytes;
   static constexpr int kOffBar = kOffV + kVStages * kTileBytes;
-  // barriers: Q, Kfull[KS], Kempty[KS], Vfull[VS], Vempty[VS], Sfull[2], Pfull[2], Odone[2], Fin
-  static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 1;
+  // barriers: Q, Kfull[KS], Kempty[KS], Vfull[VS], Vempty[VS], Sfull[2], Pfull[2][2 halves],
+  // Odone[2], Fin
+  static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 2 + 4 + 2 + 1;
   static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;   // + slack for 1 KB alignment
   static constexpr int kThreads = 384;
@@ -93,9 +94,9 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1)
   auto BAR_VF = [&](int s) { return bar0 + 8u * (1 + 2 * KS + s); };
   auto BAR_VE = [&](int s) { return bar0 + 8u * (1 + 2 * KS + VS + s); };
   auto BAR_SF = [&](int t) { return bar0 + 8u * (1 + 2 * KS + 2 * VS + t); };
-  auto BAR_PF = [&](int t) { return bar0 + 8u * (3 + 2 * KS + 2 * VS + t); };
-  auto BAR_OD = [&](int t) { return bar0 + 8u * (5 + 2 * KS + 2 * VS + t); };
-  const uint32_t BAR_FIN = bar0 + 8u * (7 + 2 * KS + 2 * VS);
+  auto BAR_PF = [&](int t, int half) { return bar0 + 8u * (3 + 2 * KS + 2 * VS + 2 * t + half); };
+  auto BAR_OD = [&](int t) { return bar0 + 8u * (7 + 2 * KS + 2 * VS + t); };
+  const uint32_t BAR_FIN = bar0 + 8u * (9 + 2 * KS + 2 * VS);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
@@ -158,7 +159,8 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(BAR_SF(t), 1);
-      mbar_init(BAR_PF(t), 128);
+      mbar_init(BAR_PF(t, 0), 4);   // one arrival per softmax warp
+      mbar_init(BAR_PF(t, 1), 4);
       mbar_init(BAR_OD(t), 1);
     }
     mbar_init(BAR_FIN, 1);
@@ -249,17 +251,22 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1)
       // O_t += P_t V_j once P_t (softmax of tile t) and V_j are ready
       // O_t += P_t V_j once P_t (softmax of tile t) is ready; V_j's arrival
       // is awaited by the caller beforehand, off the P-ready path.
-      auto issue_pv = [&](int t, int j, bool release_v) -> bool {
-        if (!mbar_wait(BAR_PF(t), j & 1, abort_flag)) return false;
-        tc_fence_after();
+      auto issue_pv = [&](int t, int j, bool release_v, bool last) -> bool {
         const int st = j % VS;
         const uint32_t tP = tmem + 256u + 128u * t;
         const uint32_t tO = tmem + 128u * t;
         const uint32_t vb = v_lo + ((st * C::kTileBytes) >> 4);
+        // P arrives in two halves of 64 keys; the first four MMAs run while
+        // the softmax still computes the second half
 #pragma unroll
-        for (int k = 0; k < kBN / 16; ++k)
-          mma_ts(tO, tP + k * 8, desc(vb + ((k * 2048) >> 4)), kIdescPV, (j > 0 || k > 0) ? 1u : 0u);
-        mma_commit(BAR_OD(t));
+        for (int half = 0; half < 2; ++half) {
+          if (!mbar_wait(BAR_PF(t, half), j & 1, abort_flag)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int k = 4 * half; k < 4 * half + 4; ++k)
+            mma_ts(tO, tP + k * 8, desc(vb + ((k * 2048) >> 4)), kIdescPV, (j > 0 || k > 0) ? 1u : 0u);
+        }
+        if (last) mma_commit(BAR_OD(t));   // single phase: O_t is final
         if (release_v) mma_commit(BAR_VE(st));
         return true;
       };
@@ -271,7 +278,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1)
         tc_fence_after();
         if (j < nt0) issue_s(0, j);
         if (j >= 1 && j - 1 < nt1) {
-          ok = issue_pv(1, j - 1, true);   // V_{j-1} arrived before O0 += P0 V_{j-1}
+          ok = issue_pv(1, j - 1, true, j - 1 == nt1 - 1);   // V_{j-1} arrived before O0 += P0 V_{j-1}
           if (!ok) break;
         }
         if (j < nt1) issue_s(1, j);
@@ -279,11 +286,11 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1)
         ok = wait_v(j);                    // V_j is needed by O0 (now) or O1 (next)
         if (!ok) break;
         if (j < nt0) {
-          ok = issue_pv(0, j, j >= nt1);   // V_j is Q0's alone when Q1 does not read it
+          ok = issue_pv(0, j, j >= nt1, j == nt0 - 1);   // V_j is Q0's alone when Q1 does not read it
           if (!ok) break;
         }
       }
-      if (ok && nt1 > 0) issue_pv(1, nt1 - 1, true);
+      if (ok && nt1 > 0) issue_pv(1, nt1 - 1, true, true);
       mma_commit(BAR_FIN);   // every MMA issued above has finished once this lands
       mbar_wait_drain(BAR_FIN, 0);
     }
@@ -341,61 +348,60 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1)
       const float alpha = grow ? ex2_approx(m - m_new) : 1.0f;
       const float2 sl22 = make_float2(sl2, sl2);
       const float2 neg2 = make_float2(-m_new, -m_new);
-      uint32_t pk[kBN / 2];
+      if (j > 0 && __any_sync(0xffffffffu, grow)) {
+        // O_t += P V of the previous key tile is complete here: that MMA was
+        // issued before the one that produced this S, the commit tracked by
+        // BAR_SF covers every MMA issued before it, and MMAs complete in issue
+        // order.  So O_t can be rescaled without another wait.
+        const float2 a2 = make_float2(alpha, alpha);
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tO + c * 32, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const float2 v = __fmul2_rn(make_float2(__uint_as_float(r[e]), __uint_as_float(r[e + 1])), a2);
+            r[e] = __float_as_uint(v.x);
+            r[e + 1] = __float_as_uint(v.y);
+          }
+          tmem_st32(tO + c * 32, r);
+        }
+      }
+      // P in two halves of 64 keys (32 packed columns each), each published
+      // as soon as it is in TMEM
       float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                        make_float2(0.f, 0.f)};
 #pragma unroll
-      for (int i = 0; i < kBN / 2; ++i) {
-        const float2 y = __ffma2_rn(x[i], sl22, neg2);
-        float2 pe;
-        if ((i & 7) < 3) {   // three pairs in eight on the FMA pipe, the rest on MUFU
-          pe = exp2_poly2(y);
-        } else {
-          pe = make_float2(ex2_approx(y.x), ex2_approx(y.y));
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+          const int i = 32 * half + u;
+          const float2 y = __ffma2_rn(x[i], sl22, neg2);
+          float2 pe;
+          if ((i & 7) < 3) {   // three pairs in eight on the FMA pipe, the rest on MUFU
+            pe = exp2_poly2(y);
+          } else {
+            pe = make_float2(ex2_approx(y.x), ex2_approx(y.y));
+          }
+          acc[i & 3] = __fadd2_rn(acc[i & 3], pe);
+          pk[u] = pack_bf16x2(pe.x, pe.y);
         }
-        acc[i & 3] = __fadd2_rn(acc[i & 3], pe);
-        pk[i] = pack_bf16x2(pe.x, pe.y);
+        tmem_st32(tS + 32 * half, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR_PF(qt, half));   // one arrival per warp
       }
       const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
       const float2 a4 = __fadd2_rn(a01, a23);
       l = l * alpha + (a4.x + a4.y);
       m = m_new;
-      if (j > 0) {
-        // O_t += P V of the previous tile must be complete before O_t is
-        // rescaled and before P overwrites S; waiting every tile keeps the
-        // barrier within one phase of this waiter.
-        ok = __all_sync(0xffffffffu, mbar_wait(BAR_OD(qt), (j - 1) & 1, abort_flag));
-        if (!ok) break;
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, grow)) {
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t r[32];
-            tmem_ld32(tO + c * 32, r);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-            tmem_st32(tO + c * 32, r);
-          }
-        }
-      }
-      {
-        uint32_t r0[32], r1[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          r0[e] = pk[e];
-          r1[e] = pk[32 + e];
-        }
-        tmem_st32(tS, r0);
-        tmem_st32(tS + 32, r1);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(BAR_PF(qt));
       iter_next(it);
     }
-    if (ok && nt > 0) {
-      ok = __all_sync(0xffffffffu, mbar_wait(BAR_OD(qt), (nt - 1) & 1, abort_flag));
+    if (ok && nt > 0) {   // BAR_OD(t) completes once, after the last O_t += P V
+      ok = __all_sync(0xffffffffu, mbar_wait(BAR_OD(qt), 0, abort_flag));
     }
     if (ok && nt > 0) {
       tc_fence_after();
