@@ -283,26 +283,23 @@ def run_gpu(args, wl):
     lse_part = torch.empty(V, hq, lq, dtype=f32, device=dev)
     ws = torch.empty(sz["workspace_bytes"], dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
-    stages = ["score", "topk", "gather", "attn", "merge"]
+    stages = ["compress", "attn", "merge"]
 
     def step(s, ev=None):
+        """One layer pass through the stage entry points, in the order and
+        with the kernels spava_layer_fwd uses: the one-launch compression
+        (query sum, scores, top-lp, passing gather), attention, merge."""
         x = sets[s % 3]
         if lp > 0:
-            spava.score(p, x["Q"], x["K"], qsum, scores, stream=stream)
-            if ev: ev[0].record(stream)
-            spava.select_topk(p, scores, idx, stream=stream)
-            if ev: ev[1].record(stream)
-            spava.gather_passing(p, x["K"], x["V"], idx, Kp, Vp, stream=stream)
-        elif ev:
-            ev[0].record(stream); ev[1].record(stream)
-        if ev: ev[2].record(stream)
+            spava.compress(p, x["Q"], x["K"], x["V"], qsum, scores, idx, Kp, Vp, stream=stream)
+        if ev: ev[0].record(stream)
         spava.attn_fwd(p, x["Q"], x["K"], x["V"], Kp if lp else None, Vp if lp else None,
                        O, lse, O_part, lse_part, stream=stream)
-        if ev: ev[3].record(stream)
+        if ev: ev[1].record(stream)
         spava.lse_merge(p, O_part, lse_part, O, lse, stream=stream)
-        if ev: ev[4].record(stream)
+        if ev: ev[2].record(stream)
 
-    launches_per_step = (4 if lp > 0 else 0) + 2   # qsum, score, topk, gather | attn, merge
+    launches_per_step = (1 if lp > 0 else 0) + 2   # compress | attn, merge
 
     for i in range(args.warmup):
         step(i)
@@ -310,7 +307,7 @@ def run_gpu(args, wl):
     assert spava.device_error() == 0
 
     # ---------------- timed region: K steps, per-stage events on the launch stream
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages))] for _ in range(args.steps)]
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     t_begin = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
@@ -410,9 +407,10 @@ def report(args, wl, sz, world, n, ms_per_step, value, stage_ms, stages, fused_m
     # algorithmic bytes of the HBM-bound stages
     S, P = sz["score_cols"], sz["passing_rows"]
     by = {
-        "score": hkv * S * d * 2 + hkv * S * 4 + lq * hq * d * 2,
-        "topk": hkv * S * 4 + (V - 1) * hkv * lp * 4,
-        "gather": 2 * 2 * P * hkv * d * 2 + (V - 1) * hkv * lp * 4,
+        # K rows of blocks 0..V-2 read once + scores written + the query block
+        # read + indices written + kept K,V rows read and written
+        "compress": hkv * S * d * 2 + hkv * S * 4 + lq * hq * d * 2 + (V - 1) * hkv * lp * 4
+                    + 2 * 2 * P * hkv * d * 2,
         "merge": V * lq * hq * (d + 1) * 4 + lq * hq * (d * 2 + 4),
     }
     stage_info = {}

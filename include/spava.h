@@ -122,6 +122,18 @@ spava_status_t spava_gather_passing(const spava_problem_t* prob, const void* K,
                                     const void* V, const int32_t* idx,
                                     void* Kp, void* Vp, spava_stream_t stream);
 
+/* Steps 1-3 fused in one launch: the same qsum, scores, idx, Kp and Vp as
+ * spava_score + spava_select_topk + spava_gather_passing ([SC] Fig. 5 caption:
+ * importance estimation, then the essential KVs).  One cluster of 8 CTAs per
+ * (block, KV head) streams K^(h) once, selects in shared memory and copies the
+ * kept rows.  Every block length must be <= 98304 (SPAVA_ERR_UNSUPPORTED
+ * otherwise; the separate stage calls have no such limit).  With lp = 0 it
+ * does nothing. */
+spava_status_t spava_compress(const spava_problem_t* prob, const void* Q,
+                              const void* K, const void* V, float* qsum,
+                              float* scores, int32_t* idx, void* Kp, void* Vp,
+                              spava_stream_t stream);
+
 /* Step 4, one launch of causal attention over mixed key segments ([PR]
  * minor comment 2: Eq. 4 key list [K_a, K_p, K^(h)]; [SC] Fig. 3 fused
  * context and query forward; Fig. 4 load balancing):

@@ -1,0 +1,272 @@
+// Fused compression: query-block sum, KV importance scores, top-lp selection
+// and the passing-buffer gather in one launch.
+//
+// "Spava ..." (sciencestack.ai), Fig. 5 caption: Q_qr K^(h)T estimates KV
+// importance and B_c^(h) are the essential KVs; "APB-V ..." (pith.science
+// review), "What carries the argument": each context block is compressed to
+// its top-lp key-value pairs ranked by Q_qr K^T and gathered by later hosts.
+//
+// One thread-block cluster of kCompressCtas CTAs per (block h < V-1, KV head):
+//   1. each CTA sums a slice of the query block's (row, head) pairs of the KV
+//      group; the slices are added in rank order through distributed shared
+//      memory, so every CTA holds the same qsum = scale * sum q;
+//   2. each CTA streams its 1/kCompressCtas slice of K^(h) once (16-byte
+//      loads) and keeps the scores, as order-preserving 32-bit keys, in
+//      shared memory (the scores are also written out);
+//   3. MSB-first radix select over the whole block: per 8-bit pass each CTA
+//      histograms its slice and the cluster adds the histograms in rank order;
+//      every CTA derives the same threshold key T and the number of copies of
+//      T to keep (lower indices first);
+//   4. a cluster-wide scan in index order gives each selected key its rank;
+//      the CTA writes the index and copies the key's K and V rows to the
+//      passing buffer.
+#pragma once
+#include <cooperative_groups.h>
+#include <cuda_bf16.h>
+
+#include "compress.cuh"
+#include "plan.hpp"
+#include "ptx.cuh"
+
+namespace spava {
+
+constexpr int kCompressCtas = 8;
+constexpr int kCompressThreads = 512;
+constexpr int kCompressMaxSlice = 12288;   // keys per CTA (block length <= 8 x this)
+
+struct CompressParams {
+  int32_t start[kMaxV];   // first sequence row of block h
+  int32_t L[kMaxV];
+  int32_t k[kMaxV];       // lp_eff(h)
+  int32_t poff[kMaxV + 1];
+  int32_t Hq, Hkv, G, lq, lp;
+  int64_t qs, la, score_cols;
+  float scale;
+};
+
+template <int D>
+__global__ void __cluster_dims__(kCompressCtas, 1, 1) __launch_bounds__(kCompressThreads, 1)
+    compress_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
+                    const __nv_bfloat16* __restrict__ V, float* __restrict__ qsum_out,
+                    float* __restrict__ scores, int32_t* __restrict__ idx,
+                    __nv_bfloat16* __restrict__ Kp, __nv_bfloat16* __restrict__ Vp,
+                    const __grid_constant__ CompressParams p) {
+  constexpr int kParts = D / 8;                           // 16-byte chunks per row
+  constexpr int kRowsPerIter = kCompressThreads / kParts;
+  extern __shared__ uint8_t dsm[];
+  uint32_t* keys = reinterpret_cast<uint32_t*>(dsm);                          // [slice]
+  int32_t* sel_j = reinterpret_cast<int32_t*>(dsm + 4 * kCompressMaxSlice);  // [slice]
+  int32_t* sel_pos = sel_j + kCompressMaxSlice;                               // [slice]
+  __shared__ float part_q[kRowsPerIter][D];
+  __shared__ float slice_q[D];
+  __shared__ float qs_full[D];
+  __shared__ uint32_t hist[256];
+  __shared__ uint32_t tot[256];
+  __shared__ uint64_t warp_tot[32];
+  __shared__ uint32_t s_prefix, s_k;
+  __shared__ uint64_t s_cta_counts;   // (eq << 32) | gt of this CTA's slice
+  __shared__ int s_nsel;
+
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = static_cast<int>(cluster.block_rank());
+  const int h = blockIdx.y, kv = blockIdx.z;
+  const int tid = threadIdx.x;
+  const int L = p.L[h], kk = p.k[h];
+  const int j0 = static_cast<int>((static_cast<int64_t>(L) * rank) / kCompressCtas);
+  const int j1 = static_cast<int>((static_cast<int64_t>(L) * (rank + 1)) / kCompressCtas);
+  const int n = j1 - j0;   // keys of this CTA's slice
+
+  // ---- 1. qsum for this KV group
+  {
+    const int total = p.lq * p.G;
+    const int r0 = static_cast<int>((static_cast<int64_t>(total) * rank) / kCompressCtas);
+    const int r1 = static_cast<int>((static_cast<int64_t>(total) * (rank + 1)) / kCompressCtas);
+    const int pc = tid % kParts, lr = tid / kParts;
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+    for (int rr = r0 + lr; rr < r1; rr += kRowsPerIter) {
+      const int i = rr / p.G, g = kv * p.G + rr % p.G;
+      const uint4 raw = *reinterpret_cast<const uint4*>(Q + ((p.qs + i) * p.Hq + g) * D + pc * 8);
+      const __nv_bfloat16* v = reinterpret_cast<const __nv_bfloat16*>(&raw);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] += __bfloat162float(v[e]);
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) part_q[lr][pc * 8 + e] = acc[e];
+    __syncthreads();
+    for (int c = tid; c < D; c += kCompressThreads) {
+      float s = 0.f;
+      for (int r = 0; r < kRowsPerIter; ++r) s += part_q[r][c];
+      slice_q[c] = s;
+    }
+    cluster.sync();
+    for (int c = tid; c < D; c += kCompressThreads) {
+      float s = 0.f;
+      for (int r = 0; r < kCompressCtas; ++r) s += cluster.map_shared_rank(slice_q, r)[c];
+      qs_full[c] = s * p.scale;
+      if (h == 0 && rank == 0) qsum_out[kv * D + c] = s * p.scale;
+    }
+    __syncthreads();
+  }
+
+  // ---- 2. scores of this slice (one pass over K)
+  {
+    const int pc = tid % kParts, lr = tid / kParts;
+    float q8[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) q8[e] = qs_full[pc * 8 + e];
+    const int64_t row0 = p.start[h] + j0;
+    float* srow = scores + static_cast<int64_t>(kv) * p.score_cols + (p.start[h] - p.la) + j0;
+    constexpr int kU = 4;
+    for (int base = 0; base < n; base += kRowsPerIter * kU) {
+      uint4 raw[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int jj = base + u * kRowsPerIter + lr;
+        raw[u] = jj < n ? __ldcs(reinterpret_cast<const uint4*>(K + ((row0 + jj) * p.Hkv + kv) * D + pc * 8))
+                        : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int jj = base + u * kRowsPerIter + lr;
+        const __nv_bfloat16* v = reinterpret_cast<const __nv_bfloat16*>(&raw[u]);
+        float dot = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) dot = fmaf(__bfloat162float(v[e]), q8[e], dot);
+#pragma unroll
+        for (int off = kParts / 2; off >= 1; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+        if (pc == 0 && jj < n) {
+          srow[jj] = dot;
+          keys[jj] = order_key(dot);
+        }
+      }
+    }
+  }
+  __syncthreads();
+
+  // ---- 3. radix select of the kk largest keys over the cluster
+  uint32_t T = 0, keq = 0;
+  const bool all = kk >= L;
+  if (!all && kk > 0) {
+    if (tid == 0) {
+      s_prefix = 0;
+      s_k = static_cast<uint32_t>(kk);
+    }
+    uint32_t mask = 0;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      for (int i = tid; i < 256; i += kCompressThreads) hist[i] = 0;
+      __syncthreads();
+      const uint32_t prefix = s_prefix;
+      for (int i = tid; i < n; i += kCompressThreads) {
+        const uint32_t key = keys[i];
+        if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+      }
+      cluster.sync();   // every CTA's histogram is complete
+      for (int b = tid; b < 256; b += kCompressThreads) {
+        uint32_t s = 0;
+        for (int r = 0; r < kCompressCtas; ++r) s += cluster.map_shared_rank(hist, r)[b];
+        tot[b] = s;
+      }
+      __syncthreads();
+      if (tid < 32) {
+        uint32_t c[8], t8 = 0;
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+          c[b] = tot[tid * 8 + b];
+          t8 += c[b];
+        }
+        uint32_t x = t8;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const uint32_t y = __shfl_down_sync(0xffffffffu, x, off);
+          if (tid + off < 32) x += y;
+        }
+        uint32_t running = x - t8;
+        const uint32_t need = s_k;
+#pragma unroll
+        for (int b = 7; b >= 0; --b) {
+          if (running < need && running + c[b] >= need) {
+            s_prefix = prefix | (static_cast<uint32_t>(tid * 8 + b) << shift);
+            s_k = need - running;
+          }
+          running += c[b];
+        }
+      }
+      cluster.sync();   // all CTAs read every histogram before any is cleared
+      mask |= 0xFFu << shift;
+    }
+    T = s_prefix;
+    keq = s_k;
+  }
+
+  // ---- 4. ranks in index order over the cluster; write idx; gather rows
+  const int chunk = (n + kCompressThreads - 1) / kCompressThreads;
+  const int i0 = min(n, tid * chunk), i1 = min(n, i0 + chunk);
+  uint32_t gt = 0, eq = 0;
+  if (!all && kk > 0) {
+    for (int i = i0; i < i1; ++i) {
+      gt += keys[i] > T;
+      eq += keys[i] == T;
+    }
+  } else if (all) {
+    gt = i1 - i0;   // every key is kept
+  }
+  const uint64_t pre = block_exclusive_scan_u64((static_cast<uint64_t>(eq) << 32) | gt, warp_tot);
+  if (tid == kCompressThreads - 1) s_cta_counts = pre + ((static_cast<uint64_t>(eq) << 32) | gt);
+  cluster.sync();   // CTA totals visible
+  uint64_t before = 0;
+  for (int r = 0; r < rank; ++r) before += *cluster.map_shared_rank(&s_cta_counts, r);
+  // global counts before this thread's chunk, and this thread's first slot in
+  // the CTA's list of selected keys (keys kept by earlier threads of the CTA)
+  uint32_t gt_pre = static_cast<uint32_t>(before + pre);
+  uint32_t eq_pre = static_cast<uint32_t>((before + pre) >> 32);
+  const uint32_t eq_cta0 = static_cast<uint32_t>(before >> 32);   // T-copies in earlier CTAs
+  const uint32_t eq_keep_cta = keq > eq_cta0 ? keq - eq_cta0 : 0u;  // still to keep from here on
+  uint32_t lsel = all ? static_cast<uint32_t>(i0)
+                      : static_cast<uint32_t>(pre) + min(static_cast<uint32_t>(pre >> 32), eq_keep_cta);
+  int32_t* out = idx + (static_cast<int64_t>(h) * p.Hkv + kv) * p.lp;
+  if (kk > 0) {
+    for (int i = i0; i < i1; ++i) {
+      const uint32_t key = keys[i];
+      int pos = -1;
+      if (all) {
+        pos = j0 + i;
+      } else if (key > T) {
+        pos = static_cast<int>(gt_pre + min(eq_pre, keq));
+        ++gt_pre;
+      } else if (key == T) {
+        if (eq_pre < keq) pos = static_cast<int>(gt_pre + eq_pre);
+        ++eq_pre;
+      }
+      if (pos >= 0) {
+        out[pos] = j0 + i;
+        sel_j[lsel] = j0 + i;
+        sel_pos[lsel] = pos;
+        ++lsel;
+      }
+    }
+  }
+  if (rank == 0)
+    for (int t = kk + tid; t < p.lp; t += kCompressThreads) out[t] = -1;
+  if (tid == kCompressThreads - 1) s_nsel = static_cast<int>(lsel);   // = the CTA's selections
+  __syncthreads();
+  const int nsel = s_nsel;
+  // gather: half a warp per row (16 lanes x 16 B = 256 B for d = 128)
+  {
+    constexpr int kLanesPerRow = kParts;
+    const int lane_in_row = tid % kLanesPerRow, row_slot = tid / kLanesPerRow;
+    const int64_t off = p.poff[h];
+    for (int s = row_slot; s < nsel; s += kRowsPerIter) {
+      const int64_t src = static_cast<int64_t>(p.start[h]) + sel_j[s];
+      const int64_t dst = off + sel_pos[s];
+      const uint4 kx = *reinterpret_cast<const uint4*>(K + (src * p.Hkv + kv) * D + lane_in_row * 8);
+      const uint4 vx = *reinterpret_cast<const uint4*>(V + (src * p.Hkv + kv) * D + lane_in_row * 8);
+      *reinterpret_cast<uint4*>(Kp + (dst * p.Hkv + kv) * D + lane_in_row * 8) = kx;
+      *reinterpret_cast<uint4*>(Vp + (dst * p.Hkv + kv) * D + lane_in_row * 8) = vx;
+    }
+  }
+  cluster.sync();   // no CTA leaves while others may still read its shared memory
+}
+
+}  // namespace spava

@@ -12,6 +12,7 @@
 #include "../../include/spava.h"
 #include "attention.cuh"
 #include "compress.cuh"
+#include "compress_fused.cuh"
 #include "merge.cuh"
 #include "plan.hpp"
 #include "ptx.cuh"
@@ -138,6 +139,56 @@ spava_status_t run_gather(const Plan& P, const void* K, const void* V, const int
     gather_kernel<128><<<static_cast<unsigned>(blocks), 256, 0, st>>>(k, v, idx, kp, vp, gp);
   else
     gather_kernel<64><<<static_cast<unsigned>(blocks), 256, 0, st>>>(k, v, idx, kp, vp, gp);
+  return last_launch();
+}
+
+bool compress_fits(const Plan& P) {
+  for (int h = 0; h < P.V - 1; ++h)
+    if ((P.L[h] + kCompressCtas - 1) / kCompressCtas > kCompressMaxSlice) return false;
+  return true;
+}
+
+// Steps 1-3 in one launch: one cluster of kCompressCtas CTAs per (block, KV head).
+spava_status_t run_compress(const Plan& P, const void* Q, const void* K, const void* V, float* qsum,
+                            float* scores, int32_t* idx, void* Kp, void* Vp, cudaStream_t st) {
+  if (P.lp == 0) return SPAVA_OK;
+  if (!Q || !K || !V || !qsum || !scores || !idx || !Kp || !Vp) return SPAVA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(Kp) || !aligned16(Vp))
+    return SPAVA_ERR_INVALID_ARG;
+  if (!compress_fits(P)) return SPAVA_ERR_UNSUPPORTED;
+  CompressParams cp;
+  std::memset(&cp, 0, sizeof(cp));
+  for (int h = 0; h < P.V; ++h) {
+    cp.start[h] = P.start[h];
+    cp.L[h] = P.L[h];
+    cp.k[h] = P.lpe[h];
+  }
+  for (int h = 0; h <= P.V; ++h) cp.poff[h] = P.poff[h];
+  cp.Hq = P.Hq;
+  cp.Hkv = P.Hkv;
+  cp.G = P.G;
+  cp.lq = P.lq;
+  cp.lp = P.lp;
+  cp.qs = P.qs;
+  cp.la = P.la;
+  cp.score_cols = P.score_cols;
+  cp.scale = P.scale;
+  const dim3 grid(kCompressCtas, P.V - 1, P.Hkv);
+  const int smem = 12 * kCompressMaxSlice;
+  const auto* q = static_cast<const __nv_bfloat16*>(Q);
+  const auto* k = static_cast<const __nv_bfloat16*>(K);
+  const auto* v = static_cast<const __nv_bfloat16*>(V);
+  auto* kp = static_cast<__nv_bfloat16*>(Kp);
+  auto* vp = static_cast<__nv_bfloat16*>(Vp);
+  if (P.d == 128) {
+    if (cudaFuncSetAttribute(compress_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return SPAVA_ERR_CUDA;
+    compress_kernel<128><<<grid, kCompressThreads, smem, st>>>(q, k, v, qsum, scores, idx, kp, vp, cp);
+  } else {
+    if (cudaFuncSetAttribute(compress_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return SPAVA_ERR_CUDA;
+    compress_kernel<64><<<grid, kCompressThreads, smem, st>>>(q, k, v, qsum, scores, idx, kp, vp, cp);
+  }
   return last_launch();
 }
 
@@ -270,6 +321,15 @@ spava_status_t spava_gather_passing(const spava_problem_t* prob, const void* K, 
   return run_gather(P, K, V, idx, Kp, Vp, reinterpret_cast<cudaStream_t>(stream));
 }
 
+spava_status_t spava_compress(const spava_problem_t* prob, const void* Q, const void* K, const void* V,
+                              float* qsum, float* scores, int32_t* idx, void* Kp, void* Vp,
+                              spava_stream_t stream) {
+  Plan P;
+  spava_status_t s = make_plan(prob, &P);
+  if (s != SPAVA_OK) return s;
+  return run_compress(P, Q, K, V, qsum, scores, idx, Kp, Vp, reinterpret_cast<cudaStream_t>(stream));
+}
+
 spava_status_t spava_attn_fwd(const spava_problem_t* prob, const void* Q, const void* K, const void* V,
                               const void* Kp, const void* Vp, void* O, float* lse, float* O_part,
                               float* lse_part, spava_stream_t stream) {
@@ -305,7 +365,9 @@ spava_status_t spava_layer_fwd(const spava_problem_t* prob, const void* Q, const
   float* O_part = reinterpret_cast<float*>(ws + P.ws_opart);
   float* lse_part = reinterpret_cast<float*>(ws + P.ws_lsepart);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (P.lp > 0) {   // with lp = 0 no later host receives anything: skip the compression
+  if (P.lp > 0 && compress_fits(P)) {   // steps 1-3 in one launch
+    if ((s = run_compress(P, Q, K, V, qsum, scores, idx, Kp, Vp, st)) != SPAVA_OK) return s;
+  } else if (P.lp > 0) {   // with lp = 0 no later host receives anything: skip the compression
     if ((s = run_score(P, Q, K, qsum, scores, st)) != SPAVA_OK) return s;
     if ((s = run_topk(P, scores, idx, st)) != SPAVA_OK) return s;
     if ((s = run_gather(P, K, V, idx, Kp, Vp, st)) != SPAVA_OK) return s;
@@ -390,7 +452,9 @@ extern "C" spava_status_t spava_layer_fwd_noalloc(const spava_problem_t* prob, c
   float* O_part = reinterpret_cast<float*>(ws + P.ws_opart);
   float* lse_part = reinterpret_cast<float*>(ws + P.ws_lsepart);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (P.lp > 0) {
+  if (P.lp > 0 && compress_fits(P)) {
+    if ((s = run_compress(P, Q, K, V, qsum, scores, idx, Kp, Vp, st)) != SPAVA_OK) return s;
+  } else if (P.lp > 0) {
     if ((s = run_score(P, Q, K, qsum, scores, st)) != SPAVA_OK) return s;
     if ((s = run_topk(P, scores, idx, st)) != SPAVA_OK) return s;
     if ((s = run_gather(P, K, V, idx, Kp, Vp, st)) != SPAVA_OK) return s;

@@ -50,6 +50,7 @@ _SIGS = {
     "spava_score": [_PP, _VP, _VP, _VP, _VP, _VP],
     "spava_select_topk": [_PP, _VP, _VP, _VP],
     "spava_gather_passing": [_PP, _VP, _VP, _VP, _VP, _VP, _VP],
+    "spava_compress": [_PP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
     "spava_attn_fwd": [_PP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
     "spava_lse_merge": [_PP, _VP, _VP, _VP, _VP, _VP],
     "spava_layer_fwd": [_PP, _VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_size_t, _VP],
@@ -174,6 +175,27 @@ def gather_passing(p: Problem, K, V, idx, Kp=None, Vp=None, stream=None):
     _check("spava_gather_passing", lib().spava_gather_passing(
         p.ref, _ptr(K), _ptr(V), _ptr(idx), _ptr(Kp), _ptr(Vp), _stream(stream)))
     return Kp, Vp
+
+
+def compress(p: Problem, Q, K, V, qsum=None, scores=None, idx=None, Kp=None, Vp=None, stream=None):
+    """Steps 1-3 in one launch (scores, top-lp indices, passing buffer)."""
+    sz, sh = _shapes(p)
+    for t, nm in ((Q, "Q"), (K, "K"), (V, "V")):
+        _need(t, torch.bfloat16, sh[nm], nm)
+    dev = Q.device
+    qsum = torch.empty(sh["qsum"], dtype=torch.float32, device=dev) if qsum is None else qsum
+    scores = torch.empty(sh["scores"], dtype=torch.float32, device=dev) if scores is None else scores
+    idx = torch.empty(sh["idx"], dtype=torch.int32, device=dev) if idx is None else idx
+    Kp = torch.empty(sh["Kp"], dtype=torch.bfloat16, device=dev) if Kp is None else Kp
+    Vp = torch.empty(sh["Kp"], dtype=torch.bfloat16, device=dev) if Vp is None else Vp
+    for t, nm, dt, k in ((qsum, "qsum", torch.float32, "qsum"), (scores, "scores", torch.float32, "scores"),
+                         (idx, "idx", torch.int32, "idx"), (Kp, "Kp", torch.bfloat16, "Kp"),
+                         (Vp, "Vp", torch.bfloat16, "Kp")):
+        _need(t, dt, sh[k], nm)
+    _check("spava_compress", lib().spava_compress(
+        p.ref, _ptr(Q), _ptr(K), _ptr(V), _ptr(qsum), _ptr(scores), _ptr(idx), _ptr(Kp), _ptr(Vp),
+        _stream(stream)))
+    return qsum, scores, idx, Kp, Vp
 
 
 def attn_fwd(p: Problem, Q, K, V, Kp, Vp, O=None, lse=None, O_part=None, lse_part=None, stream=None):

@@ -40,8 +40,8 @@ def test_full_size_layer(name):
     p = spava.Problem.from_workload(wl)
     dev = {k: inp[k].cuda() for k in ("Q", "K", "V")}
     O, lse = spava.layer_fwd(p, dev["Q"], dev["K"], dev["V"])
-    _, scores = spava.score(p, dev["Q"], dev["K"])
-    idx = to_np(spava.select_topk(p, scores))
+    _, scores, idx, _, _ = spava.compress(p, dev["Q"], dev["K"], dev["V"])   # the layer's selection
+    idx = to_np(idx)
     torch.cuda.synchronize()
     assert spava.device_error() == 0
     s_gpu = to_np(scores)

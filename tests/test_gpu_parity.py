@@ -126,6 +126,71 @@ def _oracle_passing_dev(lay, inp, ref, hkv, d):
 
 
 @pytest.mark.parametrize("name", list(CASES))
+def test_fused_compress_stage(name):
+    """Scores, top-lp indices and the passing buffer from the one-launch
+    compression against the oracle (indices exact up to near-ties; passing
+    rows exact wherever the selection is)."""
+    wl, lay, inp, ref = _case(name)
+    if wl.lp == 0:
+        pytest.skip("lp = 0 compresses nothing")
+    p = spava.Problem.from_workload(wl)
+    d = _dev(inp)
+    qsum, scores, idx, Kp, Vp = spava.compress(p, d["Q"], d["K"], d["V"])
+    torch.cuda.synchronize()
+    _no_device_error()
+    s = to_np(scores)
+    col = 0
+    for h in range(lay.V - 1):
+        r = ref["scores"][h]
+        L = lay.block_lens[h]
+        assert max_err(s[:, col:col + L], r) <= 1e-5 * np.abs(r).max() + 1e-4, f"block {h}"
+        col += L
+    swaps, affected = compare_selection(lay, ref["scores"], ref["idx"], to_np(idx))
+    Kr, Vr = oracle.gather_passing(lay, inp["K"], inp["V"], ref["idx"])
+    Kn, Vn = to_np(Kp), to_np(Vp)
+    off = 0
+    for h in range(lay.V - 1):
+        e = lay.lp_eff(h)
+        for kv in range(lay.num_kv_heads):
+            if not affected[h][kv]:
+                assert np.array_equal(Kn[off:off + e, kv], Kr[off:off + e, kv]), (h, kv)
+                assert np.array_equal(Vn[off:off + e, kv], Vr[off:off + e, kv]), (h, kv)
+        off += e
+
+
+@pytest.mark.parametrize("L,lp,seed", [(5, 2, 0), (1000, 37, 1), (4096, 512, 2), (8191, 1, 3),
+                                        (20000, 3000, 4), (12288, 12287, 5)])
+def test_fused_compress_ties_and_sizes(L, lp, seed):
+    """Keys engineered to tie exactly (only four distinct key rows, repeated
+    across every CTA slice), odd lengths and lp near L: the fused selection
+    equals the oracle's rule on the oracle's own scores (identical rows tie
+    exactly on both sides; distinct rows are far apart)."""
+    g = torch.Generator().manual_seed(seed)
+    hq, hkv, d, lq = 2, 1, 128, 3
+    la = 8
+    blocks = [L, 7]
+    n = la + sum(blocks) + lq
+    Q = torch.randn(n, hq, d, generator=g).to(torch.bfloat16)
+    K = torch.randn(n, hkv, d, generator=g).to(torch.bfloat16)
+    V = torch.randn(n, hkv, d, generator=g).to(torch.bfloat16)
+    rows = torch.randint(0, 4, (L,), generator=g)
+    K[la:la + L] = K[la:la + 4][rows]
+    lay = oracle.make_layout(1, la, blocks, lq, lp, hq, hkv, d)
+    ref_s = oracle.importance_scores(lay, Q, K, 0)[0]
+    want = oracle.top_lp(ref_s.astype(np.float32), lp)
+    p = spava.Problem(1, la, blocks, lq, lp, hq, hkv, d)
+    _, scores, idx, Kp, Vp = spava.compress(p, Q.cuda(), K.cuda(), V.cuda())
+    assert max_err(to_np(scores)[0], ref_s) <= 1e-5 * np.abs(ref_s).max() + 1e-4
+    got = to_np(idx)[0, 0]
+    e = min(lp, L)
+    assert np.array_equal(got[:e], want)
+    assert np.all(got[e:] == -1)
+    assert np.array_equal(to_np(Kp)[:e, 0], K[la + want, 0].float().numpy())
+    assert np.array_equal(to_np(Vp)[:e, 0], V[la + want, 0].float().numpy())
+    _no_device_error()
+
+
+@pytest.mark.parametrize("name", list(CASES))
 def test_attention_stage(name):
     """Attention on the oracle's passing buffer: context/anchor rows and the
     per-host query partials."""
@@ -172,10 +237,9 @@ def test_layer_fwd(name):
     On, ln = to_np(O), to_np(lse)
     affected = {h: {kv: False for kv in range(lay.num_kv_heads)} for h in range(lay.V - 1)}
     if wl.lp > 0:
-        # the layer's own selection, read back through the stage calls
-        _, scores = spava.score(p, d["Q"], d["K"])
-        idx = to_np(spava.select_topk(p, scores))
-        swaps, affected = compare_selection(lay, ref["scores"], ref["idx"], idx)
+        # the layer's own selection (the fused compression it runs)
+        _, scores, idx, _, _ = spava.compress(p, d["Q"], d["K"], d["V"])
+        swaps, affected = compare_selection(lay, ref["scores"], ref["idx"], to_np(idx))
     for r0, r1, h in [(0, lay.anchor_len, -1)] + \
             [(lay.block_starts[h], lay.block_starts[h] + lay.block_lens[h], h) for h in range(lay.V)] + \
             [(lay.query_start, lay.n, -1)]:
