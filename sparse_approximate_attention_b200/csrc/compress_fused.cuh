@@ -119,18 +119,27 @@ __global__ void __cluster_dims__(kCompressCtas, 1, 1) __launch_bounds__(kCompres
     const int64_t row0 = p.start[h] + j0;
     float* srow = scores + static_cast<int64_t>(kv) * p.score_cols + (p.start[h] - p.la) + j0;
     constexpr int kU = 4;
-    for (int base = 0; base < n; base += kRowsPerIter * kU) {
-      uint4 raw[kU];
+    constexpr int kStep = kRowsPerIter * kU;
+    auto load = [&](int base, uint4 (&raw)[kU]) {
 #pragma unroll
       for (int u = 0; u < kU; ++u) {
         const int jj = base + u * kRowsPerIter + lr;
         raw[u] = jj < n ? __ldcs(reinterpret_cast<const uint4*>(K + ((row0 + jj) * p.Hkv + kv) * D + pc * 8))
                         : make_uint4(0, 0, 0, 0);
       }
+    };
+    // software-pipelined: the next group's loads are in flight while the
+    // current group is reduced
+    uint4 cur[kU], nxt[kU];
+    load(0, nxt);
+    for (int base = 0; base < n; base += kStep) {
+#pragma unroll
+      for (int u = 0; u < kU; ++u) cur[u] = nxt[u];
+      if (base + kStep < n) load(base + kStep, nxt);
 #pragma unroll
       for (int u = 0; u < kU; ++u) {
         const int jj = base + u * kRowsPerIter + lr;
-        const __nv_bfloat16* v = reinterpret_cast<const __nv_bfloat16*>(&raw[u]);
+        const __nv_bfloat16* v = reinterpret_cast<const __nv_bfloat16*>(&cur[u]);
         float dot = 0.f;
 #pragma unroll
         for (int e = 0; e < 8; ++e) dot = fmaf(__bfloat162float(v[e]), q8[e], dot);
@@ -164,8 +173,12 @@ __global__ void __cluster_dims__(kCompressCtas, 1, 1) __launch_bounds__(kCompres
       }
       cluster.sync();   // every CTA's histogram is complete
       for (int b = tid; b < 256; b += kCompressThreads) {
+        uint32_t v[kCompressCtas];
+#pragma unroll
+        for (int r = 0; r < kCompressCtas; ++r) v[r] = cluster.map_shared_rank(hist, r)[b];   // all in flight
         uint32_t s = 0;
-        for (int r = 0; r < kCompressCtas; ++r) s += cluster.map_shared_rank(hist, r)[b];
+#pragma unroll
+        for (int r = 0; r < kCompressCtas; ++r) s += v[r];
         tot[b] = s;
       }
       __syncthreads();
