@@ -10,7 +10,7 @@ import oracle
 import sparse_approximate_attention_b200 as spava
 from sparse_approximate_attention_b200 import workloads as W
 
-from helpers import (LSE_TOL, O_TOL, compare_selection, host_affected, layout_of, max_err,
+from helpers import (LSE_TOL, O_TOL, check_rows, compare_selection, layout_of, max_err,
                      small_workload, to_np)
 
 pytestmark = pytest.mark.gpu
@@ -228,6 +228,10 @@ def test_merge_stage(name):
 
 @pytest.mark.parametrize("name", list(CASES))
 def test_layer_fwd(name):
+    """The whole layer against the oracle, every row and head.  Where the
+    layer's top-lp set differs from the oracle's only at tolerated near-ties,
+    the affected hosts' rows are compared with the oracle recomputed on the
+    layer's own selection (both selections are valid there)."""
     wl, lay, inp, ref = _case(name)
     p = spava.Problem.from_workload(wl)
     d = _dev(inp)
@@ -236,20 +240,14 @@ def test_layer_fwd(name):
     _no_device_error()
     On, ln = to_np(O), to_np(lse)
     affected = {h: {kv: False for kv in range(lay.num_kv_heads)} for h in range(lay.V - 1)}
+    sel = np.zeros((lay.V - 1, lay.num_kv_heads, wl.lp), dtype=np.int32)
     if wl.lp > 0:
         # the layer's own selection (the fused compression it runs)
         _, scores, idx, _, _ = spava.compress(p, d["Q"], d["K"], d["V"])
-        swaps, affected = compare_selection(lay, ref["scores"], ref["idx"], to_np(idx))
-    for r0, r1, h in [(0, lay.anchor_len, -1)] + \
-            [(lay.block_starts[h], lay.block_starts[h] + lay.block_lens[h], h) for h in range(lay.V)] + \
-            [(lay.query_start, lay.n, -1)]:
-        for g in range(wl.num_q_heads):
-            kv = g // lay.group
-            if h > 0 and host_affected(lay, affected, h, kv):
-                assert np.isfinite(On[r0:r1, g]).all()
-                continue
-            assert max_err(On[r0:r1, g], ref["O"][r0:r1, g]) <= O_TOL, (r0, g)
-            assert max_err(ln[g, r0:r1], ref["lse"][g, r0:r1]) <= LSE_TOL, (r0, g)
+        sel = to_np(idx)
+        swaps, affected = compare_selection(lay, ref["scores"], ref["idx"], sel)
+    check_rows(lay, inp, sel, affected, range(lay.n), list(range(wl.num_q_heads)),
+               On, ln, ref["O"], ref["lse"])
 
 
 def test_layer_is_deterministic_and_stream_ordered():

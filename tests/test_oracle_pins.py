@@ -245,19 +245,94 @@ def test_rows_fwd_matches_full_layer():
     np.testing.assert_allclose(lse, out["lse"][heads][:, r], atol=1e-13)
 
 
-def test_gather_passing_rows():
-    lay, Q, K, Vv = _small()
+def _expected_passing(lay, Q, K):
+    """Positions of the compacted passing buffer built without the oracle:
+    per block h < V-1 and KV head, the block's keys scored by a torch einsum
+    over the query block and the KV head's query heads, the lp_eff(h) largest
+    taken by torch.topk, positions ascending, blocks in host order."""
+    qs, G = lay.query_start, lay.group
+    out = [[] for _ in range(lay.num_kv_heads)]
+    for h in range(lay.V - 1):
+        s0, L, e = lay.block_starts[h], lay.block_lens[h], lay.lp_eff(h)
+        for kv in range(lay.num_kv_heads):
+            q = Q[qs:, kv * G:(kv + 1) * G].to(torch.float64)
+            s = torch.einsum("igc,jc->j", q, K[s0:s0 + L, kv].to(torch.float64)) * lay.scale
+            top = torch.sort(torch.topk(s, e).indices).values if e else torch.zeros(0, dtype=torch.long)
+            out[kv] += (top + s0).tolist()
+    return out
+
+
+def _check_gather(lay, Q, K, Vv, Kp, Vp):
+    """V carries its own position in column 0, so Vp names where each passing
+    row came from; Kp must hold the K row of that same position."""
+    want = _expected_passing(lay, Q, K)
+    for kv in range(lay.num_kv_heads):
+        got = Vp[:, kv, 0].astype(np.int64)
+        assert got.tolist() == want[kv], f"kv {kv}: passing rows {got.tolist()} != {want[kv]}"
+        assert np.array_equal(Kp[:, kv], K[torch.as_tensor(want[kv], dtype=torch.long), kv].numpy())
+
+
+def _position_coded(lay, seed=13):
+    g = torch.Generator().manual_seed(seed)
+    n, hq, hkv, d = lay.n, lay.num_q_heads, lay.num_kv_heads, lay.head_dim
+    Q = torch.randn(n, hq, d, generator=g, dtype=torch.float64)
+    K = torch.randn(n, hkv, d, generator=g, dtype=torch.float64)
+    Vv = torch.randn(n, hkv, d, generator=g, dtype=torch.float64)
+    Vv[:, :, 0] = torch.arange(n, dtype=torch.float64)[:, None]
+    return Q, K, Vv
+
+
+def test_gather_passing_against_library_topk():
+    """The compacted passing buffers (the in-HBM stand-in for the all-gather)
+    hold, for every block in host order, the rows of the lp_eff largest-scoring
+    keys, ascending -- checked on unequal blocks, no anchor, lp clamped on
+    short blocks."""
+    lay = oracle.make_layout(3, 0, [24, 7, 32, 5, 20, 9], 6, 8, 4, 2, 16)
+    Q, K, Vv = _position_coded(lay)
     _, idx = oracle.compress(lay, Q, K)
     Kp, Vp = oracle.gather_passing(lay, K, Vv, idx)
-    off = 0
-    for h in range(lay.V - 1):
-        for t in range(lay.lp_eff(h)):
-            for kv in range(lay.num_kv_heads):
-                src = lay.block_starts[h] + idx[h][kv][t]
-                assert np.array_equal(Kp[off + t, kv], K[src, kv].numpy())
-                assert np.array_equal(Vp[off + t, kv], Vv[src, kv].numpy())
-        off += lay.lp_eff(h)
-    assert off == Kp.shape[0]
+    assert Kp.shape[0] == sum(lay.lp_eff(h) for h in range(lay.V - 1)) == 8 + 7 + 8 + 5 + 8
+    _check_gather(lay, Q, K, Vv, Kp, Vp)
+
+
+def test_gather_pin_rejects_a_misordered_buffer():
+    """The pin above is sensitive to the buffer's order: the same rows with
+    the hosts' blocks in reverse order, or one block's rows rotated, fail."""
+    lay = oracle.make_layout(2, 4, [12, 9, 15, 6], 5, 5, 2, 1, 8)
+    Q, K, Vv = _position_coded(lay, seed=3)
+    _, idx = oracle.compress(lay, Q, K)
+    Kp, Vp = oracle.gather_passing(lay, K, Vv, idx)
+    _check_gather(lay, Q, K, Vv, Kp, Vp)
+    offs = np.cumsum([0] + [lay.lp_eff(h) for h in range(lay.V - 1)])
+    rev = np.concatenate([np.arange(offs[h], offs[h + 1]) for h in reversed(range(lay.V - 1))])
+    with pytest.raises(AssertionError):
+        _check_gather(lay, Q, K, Vv, Kp[rev], Vp[rev])
+    rot = np.arange(Kp.shape[0])
+    rot[offs[1]:offs[2]] = np.roll(rot[offs[1]:offs[2]], 1)
+    with pytest.raises(AssertionError):
+        _check_gather(lay, Q, K, Vv, Kp[rot], Vp[rot])
+
+
+def test_context_rows_through_the_passing_buffer():
+    """Attention of host h's context rows over [B_a, Kp rows [0, off_h), B^(h)
+    causal] -- the key list the kernel walks -- equals the oracle's rows."""
+    lay = oracle.make_layout(2, 6, [14, 11, 9, 13], 4, 5, 4, 2, 16)
+    Q, K, Vv = _position_coded(lay, seed=8)
+    out = oracle.layer_fwd(lay, Q, K, Vv)
+    Kp, Vp = oracle.gather_passing(lay, K, Vv, out["idx"])
+    off = np.cumsum([0] + [lay.lp_eff(h) for h in range(lay.V - 1)])
+    for h in range(lay.V):
+        s0, L = lay.block_starts[h], lay.block_lens[h]
+        for g in range(lay.num_q_heads):
+            kv = g // lay.group
+            k = np.concatenate([K[:lay.anchor_len, kv].numpy(), Kp[:off[h], kv], K[s0:s0 + L, kv].numpy()])
+            v = np.concatenate([Vv[:lay.anchor_len, kv].numpy(), Vp[:off[h], kv], Vv[s0:s0 + L, kv].numpy()])
+            pre = lay.anchor_len + off[h]
+            vis = np.ones((L, len(k)), dtype=bool)
+            vis[:, pre:] = np.arange(L)[None, :] <= np.arange(L)[:, None]
+            o, l = oracle.attend(Q[s0:s0 + L, g].numpy(), k, v, lay.scale, vis)
+            np.testing.assert_allclose(o, out["O"][s0:s0 + L, g], atol=1e-12)
+            np.testing.assert_allclose(l, out["lse"][g, s0:s0 + L], atol=1e-12)
 
 
 def test_flops_count_by_enumeration():
