@@ -156,7 +156,16 @@ spava_status_t spava_lse_merge(const spava_problem_t* prob, const float* O_part,
 
 /* The whole layer: steps 1-5 in order on `stream`, with every intermediate
  * carved from `workspace` (device memory, >= spava_workspace_size bytes,
- * 256-byte aligned).  Outputs O [n, Hq, d] bf16 and lse [Hq, n] fp32. */
+ * 256-byte aligned).  Outputs O [n, Hq, d] bf16 and lse [Hq, n] fp32.
+ * Two launches: the one-launch compression (steps 1-3), then attention with
+ * the merge of step 5 in the same launch (the last of the V partial CTAs of
+ * a query tile pair merges it; [SC] Fig. 5 caption: the passing-block
+ * exchange and the merge overlap the attention).  The attention launch may
+ * start while the compression runs (programmatic dependent launch): it waits
+ * for it only before reading the passing buffer.  The work list is checked
+ * before anything is launched (SPAVA_ERR_UNSUPPORTED: more than 6144 work
+ * items of two 128-row tiles).  Blocks longer than 98304 keys fall back to
+ * the three stage kernels of steps 1-3. */
 spava_status_t spava_layer_fwd(const spava_problem_t* prob, const void* Q,
                                const void* K, const void* V, void* O,
                                float* lse, void* workspace, size_t ws_bytes,
@@ -175,19 +184,29 @@ spava_status_t spava_layer_fwd(const spava_problem_t* prob, const void* Q,
  * rejected with SPAVA_ERR_WORKSPACE before anything is launched.  The call
  * allocates no device memory.  Its first call on a device looks up the
  * array's device address on that device (cudaGetSymbolAddress); make that
- * first call before any stream capture.  All calls on a device share the
- * array and it keeps the last call's contents (nothing in it needs to start
- * at zero: each call writes every byte it reads).  Calls whose work overlaps
- * on the GPU (other streams, other host threads) race on the array and give
- * wrong results: serialise them. */
+ * first call before any stream capture.  That address stays valid until the
+ * device is reset: after cudaDeviceReset the library holds a stale address,
+ * so a process that resets a device must not call this entry on it again.
+ * All calls on a device share the array and it keeps the last call's
+ * contents (nothing in it needs to start at zero: each call writes every
+ * byte it reads, and zeroes its merge counters itself).  Calls whose work
+ * overlaps on the GPU (other streams, other host threads) race on the array
+ * and give wrong results: serialise them. */
 spava_status_t spava_layer_fwd_noalloc(const spava_problem_t* prob, const void* Q,
                                        const void* K, const void* V, void* O,
                                        float* lse, spava_stream_t stream);
 
 /* Device-side error word of the current device (0 = none); synchronizes the
  * device, then clears the word.  Bit 0: a bounded wait in the attention
- * kernel gave up. */
+ * kernel gave up; bit 1: the gather met an index outside its block. */
 spava_status_t spava_device_error(uint32_t* code);
+
+/* Test hook, not part of the layer: y[i] = the 2^x approximation that the
+ * attention softmax evaluates on the FMA pipe for a share of its
+ * exponentials (a Cody-Waite split x = i + f, a cubic least-squares fit of
+ * 2^f on [-1/2, 1/2], 2^i added to the exponent; exactly 0 below -126).
+ * x, y: device float arrays of n elements, n even, 16-byte aligned. */
+spava_status_t spava_debug_exp2_poly(const float* x, float* y, int64_t n, spava_stream_t stream);
 
 /* Human-readable name of a status code (static string). */
 const char* spava_status_string(spava_status_t status);

@@ -48,6 +48,16 @@ struct AttnParams {
   int32_t n, Hq, G, lq, qs;
   float scale_log2;
   int32_t nregions, nitems;
+  // Fused merge of the query partials: one arrival counter per (query tile
+  // pair, query head), zero before the launch; the last of the V partial
+  // CTAs of a pair merges it into the query rows of O and lse.  Null: the
+  // partials are left for a separate merge.
+  int32_t* merge_count;
+  int32_t V;
+  // 1 when launched as a programmatic dependent of the compression kernel:
+  // the passing buffer and the merge counters are read only after
+  // griddepcontrol.wait.
+  int32_t pdl_wait;
   Region regions[kMaxRegions];
   uint32_t items[kMaxItems];   // (region << 20) | pair of 128-row tiles
 };
@@ -68,7 +78,7 @@ struct AttnCfg {
   // Odone[2], Fin
   static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 2 + 4 + 2 + 1;
   static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
-  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;   // + slack for 1 KB alignment
+  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;   // tmem slot, abort flag, merge flag; + 1 KB alignment slack
   static constexpr int kThreads = 384;
   static constexpr uint32_t kRegsLow = 56;     // warpgroup 0: producer, MMA issuer
   static constexpr uint32_t kRegsHigh = 224;   // warpgroups 1, 2: softmax
@@ -76,6 +86,57 @@ struct AttnCfg {
 };
 static_assert(AttnCfg<128>::kSmemBytes <= 232448, "shared memory budget");
 static_assert(AttnCfg<64>::kSmemBytes <= 232448, "shared memory budget");
+
+__device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Merge query rows [q0, q0 + nrows) of head g from the V partials:
+// lse = log sum_h exp(lse_h), O = sum_h exp(lse_h - lse) O_h.  Eight warps,
+// one row per warp at a time, D/32 columns per lane; the partials were written
+// by other CTAs of this launch, so they are read from L2 (no L1 copies).
+template <int D>
+__device__ __forceinline__ void merge_rows(const AttnParams& p, int q0, int nrows, int g, int w8, int lane) {
+  constexpr int kPer = D / 32;
+  for (int r = w8; r < nrows; r += 8) {
+    const int qi = q0 + r;
+    const float lp = lane < p.V ? __ldcg(p.lse_part + (static_cast<int64_t>(lane) * p.Hq + g) * p.lq + qi) : -INFINITY;
+    float mx = lp;
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    float e = lane < p.V ? __expf(lp - mx) : 0.f;
+    float sum = e;
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    const float lse_tot = mx + __logf(sum);
+    const float w_mine = e / sum;          // weight of partial `lane`
+    float acc[kPer];
+#pragma unroll
+    for (int c = 0; c < kPer; ++c) acc[c] = 0.f;
+    for (int hh = 0; hh < p.V; ++hh) {
+      const float w = __shfl_sync(0xffffffffu, w_mine, hh);
+      const float* src = p.O_part + ((static_cast<int64_t>(hh) * p.lq + qi) * p.Hq + g) * D + lane * kPer;
+      if (kPer == 4) {
+        const float4 o = __ldcg(reinterpret_cast<const float4*>(src));
+        acc[0] = fmaf(w, o.x, acc[0]);
+        acc[1] = fmaf(w, o.y, acc[1]);
+        acc[2] = fmaf(w, o.z, acc[2]);
+        acc[3] = fmaf(w, o.w, acc[3]);
+      } else {
+        const float2 o = __ldcg(reinterpret_cast<const float2*>(src));
+        acc[0] = fmaf(w, o.x, acc[0]);
+        acc[1] = fmaf(w, o.y, acc[1]);
+      }
+    }
+    __nv_bfloat16* dst = p.O + (static_cast<int64_t>(p.qs + qi) * p.Hq + g) * D + lane * kPer;
+    if (kPer == 4) {
+      *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]));
+    } else {
+      *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(acc[0], acc[1]);
+    }
+    if (lane == 0) p.lse[static_cast<int64_t>(g) * p.n + p.qs + qi] = lse_tot;
+  }
+}
 
 template <int D>
 __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1)
@@ -190,12 +251,17 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1)
           tma_load_3d(sQ + t * C::kTileBytes + sl * C::kSlabBytes, &p.tm_q, BAR_Q, sl * 64, head,
                       row0 + t * kBM);
       int k_issued = 0, v_issued = 0;
+      bool waited = !p.pdl_wait;
       TileIter ik = iter_begin(), iv = iter_begin();
       for (int j = 0; j <= ntk; ++j) {
         if (j < ntk) {
           const int st = j % KS;
           if (j >= KS && !mbar_wait(BAR_KE(st), ((j / KS) - 1) & 1, abort_flag)) break;
           const Seg& sg = R.seg[ik.s];
+          if (sg.src == kSrcPass && !waited) {   // the passing buffer is written by the preceding grid
+            grid_dependency_wait();
+            waited = true;
+          }
           const CUtensorMap* tk = sg.src == kSrcMain ? &p.tm_k : &p.tm_kp;
           const int krow = sg.start + ik.kt * kBN;
           mbar_arrive_expect_tx(BAR_KF(st), C::kTileBytes);
@@ -446,6 +512,26 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1)
           }
         }
         if (valid) p.lse_part[(static_cast<int64_t>(R.host) * p.Hq + head) * p.lq + qi] = lse_nat;
+      }
+    }
+    if (p.merge_count != nullptr && R.out_kind == kOutPartial) {
+      // Last-arriver merge ("APB-V ..." pith.science review, ledger: merging
+      // partial results through their lse is exact).  Every softmax thread
+      // of the CTA takes part, whatever happened above, so the named barrier
+      // always completes.
+      __threadfence();                       // this CTA's partial rows are visible device-wide
+      named_barrier_sync(1, 256);
+      int32_t* s_last = reinterpret_cast<int32_t*>(smem + C::kOffMisc + 8);
+      if (threadIdx.x == 128) {
+        if (p.pdl_wait) grid_dependency_wait();   // the counters were zeroed by the preceding grid
+        const int qpair = (row0 - p.qs) / (2 * kBM);
+        const int old = atomicAdd(p.merge_count + qpair * p.Hq + head, 1);
+        *s_last = old == p.V - 1 ? 1 : 0;
+      }
+      named_barrier_sync(1, 256);
+      if (*s_last) {
+        __threadfence();                     // every other partial of these rows is visible
+        merge_rows<D>(p, row0 - p.qs, rv0 + max(rv1, 0), head, warp - 4, lane);
       }
     }
   }

@@ -42,6 +42,10 @@ struct CompressParams {
   int32_t Hq, Hkv, G, lq, lp;
   int64_t qs, la, score_cols;
   float scale;
+  // merge counters of the attention launch that follows (zeroed here so that
+  // no separate launch is needed); null when called on its own
+  int32_t* merge_count;
+  int32_t n_merge;
 };
 
 template <int D>
@@ -71,6 +75,11 @@ __global__ void __cluster_dims__(kCompressCtas, 1, 1) __launch_bounds__(kCompres
   const int rank = static_cast<int>(cluster.block_rank());
   const int h = blockIdx.y, kv = blockIdx.z;
   const int tid = threadIdx.x;
+  // The attention launch that follows may start on the SMs this grid leaves
+  // free; it reads nothing written here before its griddepcontrol.wait.
+  if (tid == 0) grid_dependents_launch();
+  if (p.merge_count != nullptr && blockIdx.x == 0 && h == 0 && kv == 0)
+    for (int i = tid; i < p.n_merge; i += kCompressThreads) p.merge_count[i] = 0;
   const int L = p.L[h], kk = p.k[h];
   const int j0 = static_cast<int>((static_cast<int64_t>(L) * rank) / kCompressCtas);
   const int j1 = static_cast<int>((static_cast<int64_t>(L) * (rank + 1)) / kCompressCtas);

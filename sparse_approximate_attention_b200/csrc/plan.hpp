@@ -51,9 +51,11 @@ struct Plan {
   Region regions[kMaxRegions];
   int64_t pairs = 0;
   int64_t tiles = 0;
+  int64_t items = 0;   // attention work items (pairs of 128-row tiles)
+  int n_merge = 0;   // merge counters: one per (pair of 128-row query tiles, query head)
   // workspace carving (bytes from the workspace base)
   size_t ws_qsum = 0, ws_scores = 0, ws_idx = 0, ws_kp = 0, ws_vp = 0, ws_opart = 0,
-         ws_lsepart = 0, ws_total = 0;
+         ws_lsepart = 0, ws_count = 0, ws_total = 0;
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -164,6 +166,7 @@ inline spava_status_t make_plan(const spava_problem_t* p, Plan* pl) {
     const Region& R = P.regions[r];
     for (int s = 0; s < R.nseg; ++s) P.pairs += seg_pairs(R.seg[s], R.row_start, R.row_start + R.nrows);
     P.tiles += (R.nrows + kBM - 1) / kBM;
+    P.items += ((R.nrows + kBM - 1) / kBM + 1) / 2;
   }
 
   // workspace carving for the fused layer
@@ -180,6 +183,8 @@ inline spava_status_t make_plan(const spava_problem_t* p, Plan* pl) {
   P.ws_vp = carve(2ull * static_cast<size_t>(P.passing_rows) * P.Hkv * P.d);
   P.ws_opart = carve(sizeof(float) * static_cast<size_t>(P.V) * P.lq * P.Hq * P.d);
   P.ws_lsepart = carve(sizeof(float) * static_cast<size_t>(P.V) * P.Hq * P.lq);
+  P.n_merge = ((P.lq + 2 * kBM - 1) / (2 * kBM)) * P.Hq;
+  P.ws_count = carve(sizeof(int32_t) * static_cast<size_t>(P.n_merge));
   P.ws_total = off;
   return SPAVA_OK;
 }

@@ -55,16 +55,189 @@ bool make_tmap(CUtensorMap* m, const void* base, int d, int heads, int64_t rows)
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-int sm_count() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
-  return n;
-}
-
 spava_status_t last_launch() {
   return cudaGetLastError() == cudaSuccess ? SPAVA_OK : SPAVA_ERR_CUDA;
 }
+
+// ------------------------------------------------------ once per device
+// Kernel attributes (dynamic shared memory limits) and the register check of
+// the attention kernels are set up the first time a device is used, not on
+// every call.
+constexpr int kMaxDevices = 64;
+
+struct DeviceSetup {
+  bool done = false;
+  spava_status_t status = SPAVA_OK;
+  int sm_count = 148;
+};
+std::mutex g_setup_mu;
+DeviceSetup g_setup[kMaxDevices];
+
+template <int D>
+spava_status_t setup_attn() {
+  using C = AttnCfg<D>;
+  if (cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
+      cudaSuccess)
+    return SPAVA_ERR_CUDA;
+  // The kernel moves registers from warpgroup 0 to the softmax warpgroups
+  // (setmaxnreg); refuse to launch unless the launch allocation covers that
+  // split, since an uncovered increase would never be granted.
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, attn_kernel<D>) != cudaSuccess) return SPAVA_ERR_CUDA;
+  if (static_cast<long>(fa.numRegs) * C::kThreads < 128L * C::kRegsLow + 256L * C::kRegsHigh)
+    return SPAVA_ERR_UNSUPPORTED;
+  return SPAVA_OK;
+}
+
+// The current device's setup (done on first use).  Returns its status.
+spava_status_t device_setup(const DeviceSetup** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SPAVA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return SPAVA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_setup_mu);
+  DeviceSetup& s = g_setup[dev];
+  if (!s.done) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0) s.sm_count = n;
+    spava_status_t st = setup_attn<128>();
+    if (st == SPAVA_OK) st = setup_attn<64>();
+    const int csmem = 12 * kCompressMaxSlice;
+    if (st == SPAVA_OK &&
+        (cudaFuncSetAttribute(compress_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, csmem) !=
+             cudaSuccess ||
+         cudaFuncSetAttribute(compress_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, csmem) !=
+             cudaSuccess))
+      st = SPAVA_ERR_CUDA;
+    s.status = st;
+    s.done = true;
+  }
+  *out = &s;
+  return s.status;
+}
+
+int sm_count() {
+  const DeviceSetup* s = nullptr;
+  return device_setup(&s) == SPAVA_OK ? s->sm_count : 148;
+}
+
+// ------------------------------------------------------ attention launch cache
+// The attention launch's parameter block holds the work list (every 128-row
+// tile pair sorted by cost) and five tensor maps; both depend only on the
+// problem and the input pointers.  A small cache keyed by them lets repeated
+// calls on the same buffers (the common case for a layer run many times)
+// skip the sort and the encoding.
+struct AttnKey {
+  int device;
+  int32_t H, la, lq, lp, Hq, Hkv, d;
+  float scale;
+  int32_t L[kMaxV];
+  const void *Q, *K, *V, *Kp, *Vp;
+  bool operator==(const AttnKey& o) const { return std::memcmp(this, &o, sizeof(AttnKey)) == 0; }
+};
+
+struct AttnEntry {
+  AttnKey key;
+  std::unique_ptr<AttnParams> prm;
+  int grid = 0;
+  uint64_t last_use = 0;
+};
+
+constexpr int kAttnCacheSize = 8;
+std::mutex g_attn_mu;
+AttnEntry g_attn_cache[kAttnCacheSize];
+uint64_t g_attn_clock = 0;
+
+AttnKey attn_key(const Plan& P, int dev, const void* Q, const void* K, const void* V, const void* Kp,
+                 const void* Vp) {
+  AttnKey k;
+  std::memset(&k, 0, sizeof(k));   // padding included, for the byte-wise compare
+  k.device = dev;
+  k.H = P.H;
+  k.la = P.la;
+  k.lq = P.lq;
+  k.lp = P.lp;
+  k.Hq = P.Hq;
+  k.Hkv = P.Hkv;
+  k.d = P.d;
+  k.scale = P.scale;
+  for (int h = 0; h < P.V; ++h) k.L[h] = P.L[h];
+  k.Q = Q;
+  k.K = K;
+  k.V = V;
+  k.Kp = P.passing_rows > 0 ? Kp : nullptr;
+  k.Vp = P.passing_rows > 0 ? Vp : nullptr;
+  return k;
+}
+
+// Build the input-dependent part of the attention launch (work list, tensor
+// maps, regions).  Output pointers are filled in per call.
+spava_status_t build_attn(const Plan& P, const void* Q, const void* K, const void* V, const void* Kp,
+                          const void* Vp, AttnParams* prm, int* grid) {
+  std::vector<uint32_t> items;
+  spava_status_t s = make_items(P, &items);
+  if (s != SPAVA_OK) return s;
+  const int64_t g = static_cast<int64_t>(items.size()) * P.Hq;
+  if (g > 0x7FFFFFFF) return SPAVA_ERR_UNSUPPORTED;
+  std::memset(prm, 0, sizeof(AttnParams));
+  if (!make_tmap(&prm->tm_q, Q, P.d, P.Hq, P.n) || !make_tmap(&prm->tm_k, K, P.d, P.Hkv, P.n) ||
+      !make_tmap(&prm->tm_v, V, P.d, P.Hkv, P.n))
+    return SPAVA_ERR_CUDA;
+  if (P.passing_rows > 0) {
+    if (!make_tmap(&prm->tm_kp, Kp, P.d, P.Hkv, P.passing_rows) ||
+        !make_tmap(&prm->tm_vp, Vp, P.d, P.Hkv, P.passing_rows))
+      return SPAVA_ERR_CUDA;
+  } else {   // never read: no segment refers to the passing buffer
+    prm->tm_kp = prm->tm_k;
+    prm->tm_vp = prm->tm_v;
+  }
+  prm->n = static_cast<int32_t>(P.n);
+  prm->Hq = P.Hq;
+  prm->G = P.G;
+  prm->lq = P.lq;
+  prm->qs = static_cast<int32_t>(P.qs);
+  prm->V = P.V;
+  prm->scale_log2 = P.scale * 1.44269504088896340736f;
+  prm->nregions = P.nregions;
+  prm->nitems = static_cast<int32_t>(items.size());
+  for (int r = 0; r < P.nregions; ++r) prm->regions[r] = P.regions[r];
+  std::memcpy(prm->items, items.data(), items.size() * sizeof(uint32_t));
+  *grid = static_cast<int>(g);
+  return SPAVA_OK;
+}
+
+// The cached parameter block for these inputs, built on a miss.  The caller
+// holds g_attn_mu while it uses the returned entry.
+spava_status_t attn_entry(const Plan& P, const void* Q, const void* K, const void* V, const void* Kp,
+                          const void* Vp, AttnEntry** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SPAVA_ERR_CUDA;
+  const AttnKey key = attn_key(P, dev, Q, K, V, Kp, Vp);
+  AttnEntry* victim = &g_attn_cache[0];
+  for (AttnEntry& e : g_attn_cache) {
+    if (e.prm && e.key == key) {
+      e.last_use = ++g_attn_clock;
+      *out = &e;
+      return SPAVA_OK;
+    }
+    if (!e.prm || e.last_use < victim->last_use) victim = &e;
+  }
+  if (!victim->prm) victim->prm = std::make_unique<AttnParams>();
+  victim->last_use = 0;
+  victim->key = AttnKey{};   // invalid until the build succeeds
+  spava_status_t s = build_attn(P, Q, K, V, Kp, Vp, victim->prm.get(), &victim->grid);
+  if (s != SPAVA_OK) {
+    victim->prm.reset();
+    return s;
+  }
+  victim->key = key;
+  victim->last_use = ++g_attn_clock;
+  *out = victim;
+  return SPAVA_OK;
+}
+
+}  // namespace
+
+namespace {
 
 // ----------------------------------------------------------------- stages
 spava_status_t run_score(const Plan& P, const void* Q, const void* K, float* qsum, float* scores,
@@ -83,13 +256,15 @@ spava_status_t run_score(const Plan& P, const void* Q, const void* K, float* qsu
   int64_t blocks = (chunks + kScoreThreads * kScoreUnroll - 1) / (kScoreThreads * kScoreUnroll);
   blocks = std::max<int64_t>(1, std::min<int64_t>(blocks, static_cast<int64_t>(sm_count()) * 8));
   if (P.d == 128) {
-    if (smem > 48 * 1024)
-      cudaFuncSetAttribute(score_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(score_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return SPAVA_ERR_CUDA;
     score_kernel<128><<<static_cast<unsigned>(blocks), kScoreThreads, smem, st>>>(k, qsum, scores, P.la,
                                                                                   P.score_cols, P.Hkv);
   } else {
-    if (smem > 48 * 1024)
-      cudaFuncSetAttribute(score_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(score_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return SPAVA_ERR_CUDA;
     score_kernel<64><<<static_cast<unsigned>(blocks), kScoreThreads, smem, st>>>(k, qsum, scores, P.la,
                                                                                  P.score_cols, P.Hkv);
   }
@@ -148,14 +323,20 @@ bool compress_fits(const Plan& P) {
   return true;
 }
 
-// Steps 1-3 in one launch: one cluster of kCompressCtas CTAs per (block, KV head).
+// Steps 1-3 in one launch: one cluster of kCompressCtas CTAs per (block, KV
+// head).  merge_count (may be null): the following attention launch's merge
+// counters, zeroed by this launch.
 spava_status_t run_compress(const Plan& P, const void* Q, const void* K, const void* V, float* qsum,
-                            float* scores, int32_t* idx, void* Kp, void* Vp, cudaStream_t st) {
+                            float* scores, int32_t* idx, void* Kp, void* Vp, int32_t* merge_count,
+                            cudaStream_t st) {
   if (P.lp == 0) return SPAVA_OK;
   if (!Q || !K || !V || !qsum || !scores || !idx || !Kp || !Vp) return SPAVA_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(Kp) || !aligned16(Vp))
     return SPAVA_ERR_INVALID_ARG;
   if (!compress_fits(P)) return SPAVA_ERR_UNSUPPORTED;
+  const DeviceSetup* ds = nullptr;
+  spava_status_t s = device_setup(&ds);
+  if (s != SPAVA_OK) return s;
   CompressParams cp;
   std::memset(&cp, 0, sizeof(cp));
   for (int h = 0; h < P.V; ++h) {
@@ -173,6 +354,8 @@ spava_status_t run_compress(const Plan& P, const void* Q, const void* K, const v
   cp.la = P.la;
   cp.score_cols = P.score_cols;
   cp.scale = P.scale;
+  cp.merge_count = merge_count;
+  cp.n_merge = merge_count ? P.n_merge : 0;
   const dim3 grid(kCompressCtas, P.V - 1, P.Hkv);
   const int smem = 12 * kCompressMaxSlice;
   const auto* q = static_cast<const __nv_bfloat16*>(Q);
@@ -180,76 +363,58 @@ spava_status_t run_compress(const Plan& P, const void* Q, const void* K, const v
   const auto* v = static_cast<const __nv_bfloat16*>(V);
   auto* kp = static_cast<__nv_bfloat16*>(Kp);
   auto* vp = static_cast<__nv_bfloat16*>(Vp);
-  if (P.d == 128) {
-    if (cudaFuncSetAttribute(compress_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return SPAVA_ERR_CUDA;
+  if (P.d == 128)
     compress_kernel<128><<<grid, kCompressThreads, smem, st>>>(q, k, v, qsum, scores, idx, kp, vp, cp);
-  } else {
-    if (cudaFuncSetAttribute(compress_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return SPAVA_ERR_CUDA;
+  else
     compress_kernel<64><<<grid, kCompressThreads, smem, st>>>(q, k, v, qsum, scores, idx, kp, vp, cp);
-  }
   return last_launch();
 }
 
-template <int D>
-spava_status_t launch_attn(const AttnParams& prm, int grid, cudaStream_t st) {
-  using C = AttnCfg<D>;
-  if (cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
-      cudaSuccess)
-    return SPAVA_ERR_CUDA;
-  // The kernel moves registers from warpgroup 0 to the softmax warpgroups
-  // (setmaxnreg); refuse to launch unless the launch allocation covers that
-  // split, since an uncovered increase would never be granted.
-  cudaFuncAttributes fa;
-  if (cudaFuncGetAttributes(&fa, attn_kernel<D>) != cudaSuccess) return SPAVA_ERR_CUDA;
-  if (static_cast<long>(fa.numRegs) * C::kThreads < 128L * C::kRegsLow + 256L * C::kRegsHigh)
-    return SPAVA_ERR_UNSUPPORTED;
-  attn_kernel<D><<<grid, C::kThreads, C::kSmemBytes, st>>>(prm);
-  return last_launch();
-}
-
+// Attention over every row kind in one launch.  merge_count non-null: the
+// query partials are merged in the same launch (counters must be zero).
+// dependent: launched as a programmatic dependent of the kernel just before
+// it on the stream (the layer's compression), so that it can start while
+// that kernel runs; it waits for it before reading the passing buffer or the
+// counters.
 spava_status_t run_attn(const Plan& P, const void* Q, const void* K, const void* V, const void* Kp,
                         const void* Vp, void* O, float* lse, float* O_part, float* lse_part,
-                        cudaStream_t st) {
+                        int32_t* merge_count, bool dependent, cudaStream_t st) {
   if (!Q || !K || !V || !O || !lse || !O_part || !lse_part) return SPAVA_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(O_part))
     return SPAVA_ERR_INVALID_ARG;
   if (P.passing_rows > 0 && (!Kp || !Vp || !aligned16(Kp) || !aligned16(Vp))) return SPAVA_ERR_INVALID_ARG;
-  std::vector<uint32_t> items;
-  spava_status_t s = make_items(P, &items);
+  if (P.items > kMaxItems) return SPAVA_ERR_UNSUPPORTED;
+  const DeviceSetup* ds = nullptr;
+  spava_status_t s = device_setup(&ds);
   if (s != SPAVA_OK) return s;
-  auto prm = std::make_unique<AttnParams>();
-  std::memset(prm.get(), 0, sizeof(AttnParams));
-  if (!make_tmap(&prm->tm_q, Q, P.d, P.Hq, P.n) || !make_tmap(&prm->tm_k, K, P.d, P.Hkv, P.n) ||
-      !make_tmap(&prm->tm_v, V, P.d, P.Hkv, P.n))
-    return SPAVA_ERR_CUDA;
-  if (P.passing_rows > 0) {
-    if (!make_tmap(&prm->tm_kp, Kp, P.d, P.Hkv, P.passing_rows) ||
-        !make_tmap(&prm->tm_vp, Vp, P.d, P.Hkv, P.passing_rows))
-      return SPAVA_ERR_CUDA;
-  } else {   // never read: no segment refers to the passing buffer
-    prm->tm_kp = prm->tm_k;
-    prm->tm_vp = prm->tm_v;
+  std::lock_guard<std::mutex> lock(g_attn_mu);
+  AttnEntry* e = nullptr;
+  if ((s = attn_entry(P, Q, K, V, Kp, Vp, &e)) != SPAVA_OK) return s;
+  AttnParams& prm = *e->prm;
+  prm.O = static_cast<__nv_bfloat16*>(O);
+  prm.lse = lse;
+  prm.O_part = O_part;
+  prm.lse_part = lse_part;
+  prm.merge_count = merge_count;
+  prm.pdl_wait = dependent ? 1 : 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(e->grid));
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = dependent ? 1 : 0;
+  if (P.d == 128) {
+    cfg.blockDim = dim3(AttnCfg<128>::kThreads);
+    cfg.dynamicSmemBytes = AttnCfg<128>::kSmemBytes;
+    if (cudaLaunchKernelEx(&cfg, attn_kernel<128>, prm) != cudaSuccess) return SPAVA_ERR_CUDA;
+  } else {
+    cfg.blockDim = dim3(AttnCfg<64>::kThreads);
+    cfg.dynamicSmemBytes = AttnCfg<64>::kSmemBytes;
+    if (cudaLaunchKernelEx(&cfg, attn_kernel<64>, prm) != cudaSuccess) return SPAVA_ERR_CUDA;
   }
-  prm->O = static_cast<__nv_bfloat16*>(O);
-  prm->lse = lse;
-  prm->O_part = O_part;
-  prm->lse_part = lse_part;
-  prm->n = static_cast<int32_t>(P.n);
-  prm->Hq = P.Hq;
-  prm->G = P.G;
-  prm->lq = P.lq;
-  prm->qs = static_cast<int32_t>(P.qs);
-  prm->scale_log2 = P.scale * 1.44269504088896340736f;
-  prm->nregions = P.nregions;
-  prm->nitems = static_cast<int32_t>(items.size());
-  for (int r = 0; r < P.nregions; ++r) prm->regions[r] = P.regions[r];
-  std::memcpy(prm->items, items.data(), items.size() * sizeof(uint32_t));
-  const int64_t grid = static_cast<int64_t>(items.size()) * P.Hq;
-  if (grid > 0x7FFFFFFF) return SPAVA_ERR_UNSUPPORTED;
-  return P.d == 128 ? launch_attn<128>(*prm, static_cast<int>(grid), st)
-                    : launch_attn<64>(*prm, static_cast<int>(grid), st);
+  return last_launch();
 }
 
 spava_status_t run_merge(const Plan& P, const float* O_part, const float* lse_part, void* O, float* lse,
@@ -265,6 +430,58 @@ spava_status_t run_merge(const Plan& P, const float* O_part, const float* lse_pa
     merge_kernel<64><<<static_cast<unsigned>(blocks), 256, 0, st>>>(O_part, lse_part, o, lse, P.V, P.lq, P.Hq,
                                                                    P.qs, P.n);
   return last_launch();
+}
+
+// The whole layer with its intermediates carved from `ws` (P.ws_total bytes,
+// 256-byte aligned): compression (one launch, or the three stage kernels for
+// blocks too long for it), then attention with the query-partial merge in
+// the same launch, started as a programmatic dependent of the compression.
+// The work list is built (and checked) before anything is launched.
+spava_status_t run_layer(const Plan& P, uint8_t* ws, const void* Q, const void* K, const void* V, void* O,
+                         float* lse, cudaStream_t st) {
+  float* qsum = reinterpret_cast<float*>(ws + P.ws_qsum);
+  float* scores = reinterpret_cast<float*>(ws + P.ws_scores);
+  int32_t* idx = reinterpret_cast<int32_t*>(ws + P.ws_idx);
+  void* Kp = ws + P.ws_kp;
+  void* Vp = ws + P.ws_vp;
+  float* O_part = reinterpret_cast<float*>(ws + P.ws_opart);
+  float* lse_part = reinterpret_cast<float*>(ws + P.ws_lsepart);
+  int32_t* count = reinterpret_cast<int32_t*>(ws + P.ws_count);
+  spava_status_t s;
+  if (P.items > kMaxItems) return SPAVA_ERR_UNSUPPORTED;   // before any CUDA call
+  {   // validate the attention launch first (work list, tensor maps)
+    const DeviceSetup* ds = nullptr;
+    if ((s = device_setup(&ds)) != SPAVA_OK) return s;
+    std::lock_guard<std::mutex> lock(g_attn_mu);
+    AttnEntry* e = nullptr;
+    if ((s = attn_entry(P, Q, K, V, Kp, Vp, &e)) != SPAVA_OK) return s;
+  }
+  bool dependent = false;
+  if (P.lp > 0 && compress_fits(P)) {   // steps 1-3 in one launch; it also zeroes the merge counters
+    if ((s = run_compress(P, Q, K, V, qsum, scores, idx, Kp, Vp, count, st)) != SPAVA_OK) return s;
+    dependent = true;
+  } else {
+    if (P.lp > 0) {   // with lp = 0 no later host receives anything: no compression
+      if ((s = run_score(P, Q, K, qsum, scores, st)) != SPAVA_OK) return s;
+      if ((s = run_topk(P, scores, idx, st)) != SPAVA_OK) return s;
+      if ((s = run_gather(P, K, V, idx, Kp, Vp, st)) != SPAVA_OK) return s;
+    }
+    if (cudaMemsetAsync(count, 0, sizeof(int32_t) * static_cast<size_t>(P.n_merge), st) != cudaSuccess)
+      return SPAVA_ERR_CUDA;
+  }
+  return run_attn(P, Q, K, V, Kp, Vp, O, lse, O_part, lse_part, count, dependent, st);
+}
+
+}  // namespace
+
+namespace {
+
+// y[i] = the attention softmax's FMA-pipe 2^x (exp2_poly2) applied to x[i];
+// n even.  Test hook for the approximation's error bound.
+__global__ void exp2_poly_kernel(const float2* __restrict__ x, float2* __restrict__ y, int64_t npairs) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < npairs;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    y[i] = exp2_poly2(x[i]);
 }
 
 }  // namespace
@@ -327,7 +544,7 @@ spava_status_t spava_compress(const spava_problem_t* prob, const void* Q, const 
   Plan P;
   spava_status_t s = make_plan(prob, &P);
   if (s != SPAVA_OK) return s;
-  return run_compress(P, Q, K, V, qsum, scores, idx, Kp, Vp, reinterpret_cast<cudaStream_t>(stream));
+  return run_compress(P, Q, K, V, qsum, scores, idx, Kp, Vp, nullptr, reinterpret_cast<cudaStream_t>(stream));
 }
 
 spava_status_t spava_attn_fwd(const spava_problem_t* prob, const void* Q, const void* K, const void* V,
@@ -336,7 +553,8 @@ spava_status_t spava_attn_fwd(const spava_problem_t* prob, const void* Q, const 
   Plan P;
   spava_status_t s = make_plan(prob, &P);
   if (s != SPAVA_OK) return s;
-  return run_attn(P, Q, K, V, Kp, Vp, O, lse, O_part, lse_part, reinterpret_cast<cudaStream_t>(stream));
+  return run_attn(P, Q, K, V, Kp, Vp, O, lse, O_part, lse_part, nullptr, false,
+                  reinterpret_cast<cudaStream_t>(stream));
 }
 
 spava_status_t spava_lse_merge(const spava_problem_t* prob, const float* O_part, const float* lse_part,
@@ -356,24 +574,7 @@ spava_status_t spava_layer_fwd(const spava_problem_t* prob, const void* Q, const
   if (!Q || !K || !V || !O || !lse) return SPAVA_ERR_INVALID_ARG;
   if (!workspace || ws_bytes < P.ws_total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return SPAVA_ERR_WORKSPACE;
-  auto* ws = static_cast<uint8_t*>(workspace);
-  float* qsum = reinterpret_cast<float*>(ws + P.ws_qsum);
-  float* scores = reinterpret_cast<float*>(ws + P.ws_scores);
-  int32_t* idx = reinterpret_cast<int32_t*>(ws + P.ws_idx);
-  void* Kp = ws + P.ws_kp;
-  void* Vp = ws + P.ws_vp;
-  float* O_part = reinterpret_cast<float*>(ws + P.ws_opart);
-  float* lse_part = reinterpret_cast<float*>(ws + P.ws_lsepart);
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (P.lp > 0 && compress_fits(P)) {   // steps 1-3 in one launch
-    if ((s = run_compress(P, Q, K, V, qsum, scores, idx, Kp, Vp, st)) != SPAVA_OK) return s;
-  } else if (P.lp > 0) {   // with lp = 0 no later host receives anything: skip the compression
-    if ((s = run_score(P, Q, K, qsum, scores, st)) != SPAVA_OK) return s;
-    if ((s = run_topk(P, scores, idx, st)) != SPAVA_OK) return s;
-    if ((s = run_gather(P, K, V, idx, Kp, Vp, st)) != SPAVA_OK) return s;
-  }
-  if ((s = run_attn(P, Q, K, V, Kp, Vp, O, lse, O_part, lse_part, st)) != SPAVA_OK) return s;
-  return run_merge(P, O_part, lse_part, O, lse, st);
+  return run_layer(P, static_cast<uint8_t*>(workspace), Q, K, V, O, lse, reinterpret_cast<cudaStream_t>(stream));
 }
 
 spava_status_t spava_device_error(uint32_t* code) {
@@ -384,6 +585,16 @@ spava_status_t spava_device_error(uint32_t* code) {
   if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess) return SPAVA_ERR_CUDA;
   *code = v;
   return SPAVA_OK;
+}
+
+spava_status_t spava_debug_exp2_poly(const float* x, float* y, int64_t n, spava_stream_t stream) {
+  if (!x || !y || n < 0 || (n & 1) || !aligned16(x) || !aligned16(y)) return SPAVA_ERR_INVALID_ARG;
+  if (n == 0) return SPAVA_OK;
+  const int64_t npairs = n / 2;
+  const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((npairs + 255) / 256, 148 * 8));
+  exp2_poly_kernel<<<static_cast<unsigned>(blocks), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const float2*>(x), reinterpret_cast<float2*>(y), npairs);
+  return last_launch();
 }
 
 const char* spava_status_string(spava_status_t status) {
@@ -401,16 +612,15 @@ const char* spava_status_string(spava_status_t status) {
 }  // extern "C"
 
 // ======================================================= no-allocation entry
-// A copy of the layer's sequencing whose intermediates live in a fixed
-// device array of this library instead of a caller-provided workspace.
+// The layer with its intermediates in a fixed device array of this library
+// instead of a caller-provided workspace (same sequencing: run_layer).
 namespace {
 
 constexpr size_t kStaticScratchBytes = size_t(64) << 20;   // 64 MiB per device
 __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
 
-constexpr int kMaxScratchDevices = 64;
 std::mutex g_static_scratch_mu;
-void* g_static_scratch_addr[kMaxScratchDevices] = {};
+void* g_static_scratch_addr[kMaxDevices] = {};
 
 // Device address of g_static_scratch on the current device.  The first call
 // on a device looks it up (cudaGetSymbolAddress, with that device current)
@@ -418,7 +628,7 @@ void* g_static_scratch_addr[kMaxScratchDevices] = {};
 spava_status_t static_scratch_address(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return SPAVA_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxScratchDevices) return SPAVA_ERR_UNSUPPORTED;
+  if (dev < 0 || dev >= kMaxDevices) return SPAVA_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_static_scratch_mu);
   if (!g_static_scratch_addr[dev]) {
     void* p = nullptr;
@@ -441,24 +651,8 @@ extern "C" spava_status_t spava_layer_fwd_noalloc(const spava_problem_t* prob, c
   if (!Q || !K || !V || !O || !lse) return SPAVA_ERR_INVALID_ARG;
   void* base = nullptr;
   if ((s = static_scratch_address(&base)) != SPAVA_OK) return s;
-  // Every byte the steps below read from the scratch is written earlier in
-  // the same call, so nothing has to be cleared between calls.
-  auto* ws = static_cast<uint8_t*>(base);
-  float* qsum = reinterpret_cast<float*>(ws + P.ws_qsum);
-  float* scores = reinterpret_cast<float*>(ws + P.ws_scores);
-  int32_t* idx = reinterpret_cast<int32_t*>(ws + P.ws_idx);
-  void* Kp = ws + P.ws_kp;
-  void* Vp = ws + P.ws_vp;
-  float* O_part = reinterpret_cast<float*>(ws + P.ws_opart);
-  float* lse_part = reinterpret_cast<float*>(ws + P.ws_lsepart);
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (P.lp > 0 && compress_fits(P)) {
-    if ((s = run_compress(P, Q, K, V, qsum, scores, idx, Kp, Vp, st)) != SPAVA_OK) return s;
-  } else if (P.lp > 0) {
-    if ((s = run_score(P, Q, K, qsum, scores, st)) != SPAVA_OK) return s;
-    if ((s = run_topk(P, scores, idx, st)) != SPAVA_OK) return s;
-    if ((s = run_gather(P, K, V, idx, Kp, Vp, st)) != SPAVA_OK) return s;
-  }
-  if ((s = run_attn(P, Q, K, V, Kp, Vp, O, lse, O_part, lse_part, st)) != SPAVA_OK) return s;
-  return run_merge(P, O_part, lse_part, O, lse, st);
+  // Every byte the layer reads from the scratch is written earlier in the
+  // same call (the merge counters are zeroed by the call itself), so nothing
+  // has to be cleared between calls.
+  return run_layer(P, static_cast<uint8_t*>(base), Q, K, V, O, lse, reinterpret_cast<cudaStream_t>(stream));
 }

@@ -55,6 +55,8 @@ _SIGS = {
     "spava_lse_merge": [_PP, _VP, _VP, _VP, _VP, _VP],
     "spava_layer_fwd": [_PP, _VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_size_t, _VP],
     "spava_device_error": [ctypes.POINTER(ctypes.c_uint32)],
+    "spava_layer_fwd_noalloc": [_PP, _VP, _VP, _VP, _VP, _VP, _VP],
+    "spava_debug_exp2_poly": [_VP, _VP, ctypes.c_int64, _VP],
 }
 
 
@@ -271,9 +273,17 @@ def layer_fwd_noalloc(p: Problem, Q, K, V, O, lse, stream=None):
     for t, nm in ((Q, "Q"), (K, "K"), (V, "V"), (O, "O")):
         _need(t, torch.bfloat16, sh[nm], nm)
     _need(lse, torch.float32, sh["lse"], "lse")
-    f = lib().spava_layer_fwd_noalloc
-    f.argtypes = [_PP, _VP, _VP, _VP, _VP, _VP, _VP]
-    f.restype = ctypes.c_int
-    _check("spava_layer_fwd_noalloc", f(p.ref, _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(lse),
-                                        _stream(stream)))
+    _check("spava_layer_fwd_noalloc", lib().spava_layer_fwd_noalloc(
+        p.ref, _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(lse), _stream(stream)))
     return O, lse
+
+
+def debug_exp2_poly(x, y=None, stream=None):
+    """The attention softmax's FMA-pipe 2^x approximation applied to x
+    (float32, even length, on the GPU) -- a test hook for its error bound."""
+    if x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous() or x.numel() % 2:
+        raise ValueError("x: expected a contiguous cuda float32 tensor of even length")
+    y = torch.empty_like(x) if y is None else y
+    _need(y, torch.float32, tuple(x.shape), "y")
+    _check("spava_debug_exp2_poly", lib().spava_debug_exp2_poly(_ptr(x), _ptr(y), x.numel(), _stream(stream)))
+    return y

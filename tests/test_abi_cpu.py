@@ -102,6 +102,13 @@ def test_null_problem_and_null_block_lens():
 
 
 def test_too_many_tiles_is_unsupported_not_a_crash():
-    p = spava.Problem(16, 0, [32768] * 32, 16, 16, 2, 1, 128)   # ~1M rows -> > 6144 tiles
+    """A layer whose attention work list exceeds the launch's capacity is
+    refused before anything is launched or dereferenced (the pointers below
+    are never touched; no GPU is needed)."""
+    p = spava.Problem(16, 0, [65536] * 32, 16, 16, 2, 1, 128)   # ~2M rows -> > 6144 work items
     sz = p.sizes()
-    assert sz["attn_tiles"] > 6144
+    assert sz["attn_tiles"] > 2 * 6144
+    fake = ctypes.c_void_p(1 << 20)   # 256-byte aligned, never dereferenced
+    r = spava.lib().spava_layer_fwd(p.ref, fake, fake, fake, fake, fake, fake,
+                                    ctypes.c_size_t(sz["workspace_bytes"]), None)
+    assert r == 2   # SPAVA_ERR_UNSUPPORTED

@@ -286,3 +286,35 @@ def test_bad_arguments_are_rejected_before_launch():
                            ctypes.c_void_p(ws.data_ptr()), ctypes.c_void_p(ws.data_ptr()), None)
     assert r == 1              # misaligned Q
     _no_device_error()
+
+
+def test_layer_long_block_fallback():
+    """A context block longer than the one-launch compression takes (98304
+    keys): the layer runs the three stage kernels for steps 1-3 instead, then
+    the same attention launch.  Scores and indices are checked in full, rows
+    on samples the oracle computes one by one."""
+    wl = small_workload("long_block", 16, (100000, 64), 8, 128, 2, 1, 64, seed=9)
+    lay = layout_of(wl)
+    inp = W.make_inputs(wl)
+    p = spava.Problem.from_workload(wl)
+    d = _dev(inp)
+    O, lse = spava.layer_fwd(p, d["Q"], d["K"], d["V"])
+    _, scores = spava.score(p, d["Q"], d["K"])              # the stage kernels the layer ran
+    idx = to_np(spava.select_topk(p, scores))
+    torch.cuda.synchronize()
+    _no_device_error()
+    ref_scores, ref_idx = oracle.compress(lay, inp["Q"], inp["K"])
+    s = to_np(scores)
+    assert max_err(s[:, :100000], ref_scores[0]) <= 1e-5 * np.abs(ref_scores[0]).max() + 1e-4
+    swaps, affected = compare_selection(lay, ref_scores, ref_idx, idx)
+    s0 = lay.block_starts[0]
+    rng = np.random.default_rng(3)
+    rows = list(range(16)) + list(range(s0, s0 + 16)) + list(range(s0 + 100000 - 16, s0 + 100000)) + \
+        sorted(set(int(x) for x in rng.integers(s0, s0 + 100000, 16))) + \
+        list(range(lay.block_starts[1], lay.block_starts[1] + 64)) + list(range(lay.query_start, lay.n))
+    heads = [0, 1]
+    got_rows, o_ref, l_ref = oracle.rows_fwd(lay, inp["Q"], inp["K"], inp["V"], ref_idx, rows, heads)
+    r = torch.as_tensor(got_rows).cuda()
+    On = O[r][:, heads].float().cpu().numpy().astype(np.float64)
+    Ln = lse[heads][:, r].cpu().numpy()
+    check_rows(lay, inp, idx, affected, got_rows, heads, On, Ln, o_ref, l_ref)

@@ -37,17 +37,24 @@ def _case(wl):
     return p, Q, K, V
 
 
-def test_noalloc_matches_workspace_entry_on_two_calls_in_a_row():
+def test_noalloc_matches_workspace_entry_on_calls_in_a_row():
+    """Three calls in a row on different problems: a larger one, a smaller
+    one, then one with lp = 0 (no compression: attention reads no passing
+    rows from the shared array), the last through the Python wrapper."""
     cases = [W.Workload("frames_small", 2, 256, [1024, 777, 1024, 300], 128, 256, 8, 2, 128,
                         generator="frames", seed=77),
-             W.workloads()["tiny"]]
-    for wl in cases:                     # call 1 (larger problem), then call 2 (smaller)
+             W.workloads()["tiny"],
+             W.Workload("no_passing", 2, 40, [300, 129, 256, 77], 20, 0, 4, 2, 128, seed=78)]
+    for n_call, wl in enumerate(cases):
         p, Q, K, V = _case(wl)
         n = Q.shape[0]
         O_ref, lse_ref = spava.layer_fwd(p, Q, K, V)
         O = torch.full_like(Q, float("nan"))
         lse = torch.full((wl.num_q_heads, n), float("nan"), device="cuda")
-        assert _noalloc(p, Q, K, V, O, lse) == 0
+        if n_call < 2:
+            assert _noalloc(p, Q, K, V, O, lse) == 0
+        else:
+            spava.layer_fwd_noalloc(p, Q, K, V, O, lse)
         torch.cuda.synchronize()
         assert spava.device_error() == 0
         assert torch.isfinite(O.float()).all() and torch.isfinite(lse).all()
