@@ -126,7 +126,7 @@ spava_status_t spava_gather_passing(const spava_problem_t* prob, const void* K,
  * spava_score + spava_select_topk + spava_gather_passing ([SC] Fig. 5 caption:
  * importance estimation, then the essential KVs).  One cluster of 8 CTAs per
  * (block, KV head) streams K^(h) once, selects in shared memory and copies the
- * kept rows.  Every block length must be <= 98304 (SPAVA_ERR_UNSUPPORTED
+ * kept rows.  Every block length must be <= 24576 (SPAVA_ERR_UNSUPPORTED
  * otherwise; the separate stage calls have no such limit).  With lp = 0 it
  * does nothing. */
 spava_status_t spava_compress(const spava_problem_t* prob, const void* Q,
@@ -164,7 +164,7 @@ spava_status_t spava_lse_merge(const spava_problem_t* prob, const float* O_part,
  * start while the compression runs (programmatic dependent launch): it waits
  * for it only before reading the passing buffer.  The work list is checked
  * before anything is launched (SPAVA_ERR_UNSUPPORTED: more than 6144 work
- * items of two 128-row tiles).  Blocks longer than 98304 keys fall back to
+ * items of two 128-row tiles).  Blocks longer than 24576 keys fall back to
  * the three stage kernels of steps 1-3. */
 spava_status_t spava_layer_fwd(const spava_problem_t* prob, const void* Q,
                                const void* K, const void* V, void* O,

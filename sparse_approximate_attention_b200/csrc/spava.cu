@@ -101,7 +101,7 @@ spava_status_t device_setup(const DeviceSetup** out) {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0) s.sm_count = n;
     spava_status_t st = setup_attn<128>();
     if (st == SPAVA_OK) st = setup_attn<64>();
-    const int csmem = 12 * kCompressMaxSlice;
+    const int csmem = compress_smem_bytes(kCompressMaxBlock);
     if (st == SPAVA_OK &&
         (cudaFuncSetAttribute(compress_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, csmem) !=
              cudaSuccess ||
@@ -319,7 +319,7 @@ spava_status_t run_gather(const Plan& P, const void* K, const void* V, const int
 
 bool compress_fits(const Plan& P) {
   for (int h = 0; h < P.V - 1; ++h)
-    if ((P.L[h] + kCompressCtas - 1) / kCompressCtas > kCompressMaxSlice) return false;
+    if (P.L[h] > kCompressMaxBlock) return false;
   return true;
 }
 
@@ -356,8 +356,9 @@ spava_status_t run_compress(const Plan& P, const void* Q, const void* K, const v
   cp.scale = P.scale;
   cp.merge_count = merge_count;
   cp.n_merge = merge_count ? P.n_merge : 0;
+  for (int h = 0; h < P.V - 1; ++h) cp.lmax = std::max(cp.lmax, P.L[h]);
   const dim3 grid(kCompressCtas, P.V - 1, P.Hkv);
-  const int smem = 12 * kCompressMaxSlice;
+  const int smem = compress_smem_bytes(cp.lmax);   // sized to the longest block: two CTAs per SM fit
   const auto* q = static_cast<const __nv_bfloat16*>(Q);
   const auto* k = static_cast<const __nv_bfloat16*>(K);
   const auto* v = static_cast<const __nv_bfloat16*>(V);

@@ -289,7 +289,7 @@ def test_bad_arguments_are_rejected_before_launch():
 
 
 def test_layer_long_block_fallback():
-    """A context block longer than the one-launch compression takes (98304
+    """A context block longer than the one-launch compression takes (24576
     keys): the layer runs the three stage kernels for steps 1-3 instead, then
     the same attention launch.  Scores and indices are checked in full, rows
     on samples the oracle computes one by one."""
