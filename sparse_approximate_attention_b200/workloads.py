@@ -26,6 +26,7 @@ FRAME_TOKENS = 1024   # tokens per video frame in the long-video generator
 FRAME_RANK = 16       # rank of the per-frame key/value embedding
 NOISE = 0.3           # isotropic noise added to the low-rank frame part
 QR_HIT_FRACTION = 0.02  # fraction of context keys the text query correlates with
+TEXT_NEEDLES = 16       # needle keys per KV head in the text generator
 
 
 @dataclass
@@ -47,7 +48,7 @@ class Workload:
     num_q_heads: int
     num_kv_heads: int
     head_dim: int
-    generator: str = "gaussian"       # "gaussian" | "needles" | "frames"
+    generator: str = "gaussian"       # "gaussian" | "needles" | "frames" | "text"
     seed: int = 0
     description: str = ""
     extra: Dict = field(default_factory=dict)
@@ -117,6 +118,16 @@ def workloads() -> Dict[str, Workload]:
         generator="frames", seed=1240,
         description="half of the 3B-shaped layer (H=2/V=4, anchor 1024 + 4x8192 + "
         "query 128, lp=1024): the profiling case, inputs still larger than L2")
+    # long-context text prefill in the shape of the pages' RULER transfer
+    # setting: Llama-3.1-8B attention (32 query heads, 8 KV heads, d = 128),
+    # 128K input on 8 hosts (16 virtual hosts), la = n/64, lp = n/128 (the
+    # ledger's defaults), a 256-token question block
+    w["ruler_llama31_8b_128k"] = Workload(
+        "ruler_llama31_8b_128k", num_hosts=8, anchor_len=2048, block_lens=[8048] * 16,
+        query_len=256, lp=1024, num_q_heads=32, num_kv_heads=8, head_dim=128,
+        generator="text", seed=1241,
+        description="RULER-shaped text prefill, Llama-3.1-8B attention, n = 131072, H=8/V=16, "
+        "anchor 2048 + 16x8048 + query 256, lp = 1024")
     blens = _unequal_blocks(1239, 8, 65536, 4096, 12288)
     w["exact_dense_3b_unequal"] = Workload(
         "exact_dense_3b_unequal", num_hosts=4, anchor_len=1024, block_lens=blens,
@@ -147,6 +158,11 @@ def make_inputs(wl: Workload, seed: Optional[int] = None) -> Dict[str, torch.Ten
               block's queries correlate with a random 2% subset T of the
               context keys of their KV head: q = 0.8 k_t + 0.6 N(0,1) with
               t drawn uniformly from T.
+    text    : Q, K, V ~ N(0,1) (a needle-in-a-haystack item's shape): per KV
+              head, TEXT_NEEDLES context positions hold needle keys; each
+              query-block query is 0.8 k_t + 0.6 N(0,1) with t drawn from that
+              head's needles, so the question points at a few keys spread over
+              the whole context.
     """
     seed = wl.seed if seed is None else seed
     g = torch.Generator().manual_seed(seed)
@@ -176,6 +192,21 @@ def make_inputs(wl: Workload, seed: Optional[int] = None) -> Dict[str, torch.Ten
                    V=V.to(torch.bfloat16))
         return out
 
+    if wl.generator == "text":
+        Q = _randn(g, n, hq, d)
+        K = _randn(g, n, hkv, d)
+        V = _randn(g, n, hkv, d)
+        nctx = ctx1 - ctx0
+        needles = []
+        for kv in range(hkv):
+            pos = torch.randperm(nctx, generator=g)[:TEXT_NEEDLES] + ctx0
+            needles.append(pos)
+            for gg in range(kv * grp, (kv + 1) * grp):
+                pick = pos[torch.randint(0, len(pos), (lq,), generator=g)]
+                Q[ctx1:, gg, :] = 0.8 * K[pick, kv, :] + 0.6 * _randn(g, lq, d)
+        out.update(Q=Q.to(torch.bfloat16), K=K.to(torch.bfloat16), V=V.to(torch.bfloat16),
+                   needle_positions=torch.stack(needles))
+        return out
     if wl.generator != "frames":
         raise ValueError(wl.generator)
     Q = torch.empty(n, hq, d, dtype=torch.bfloat16)

@@ -17,7 +17,7 @@ from helpers import check_rows, compare_selection, layout_of, max_err, to_np
 pytestmark = pytest.mark.gpu
 
 FULL = ["qwen25vl3b_64f", "qwen25vl7b_128k", "longvideo_256k_lp512", "longvideo_256k_lp2048",
-        "longvideo_256k_lp4096", "exact_dense_3b", "exact_dense_3b_unequal"]
+        "longvideo_256k_lp4096", "exact_dense_3b", "exact_dense_3b_unequal", "ruler_llama31_8b_128k"]
 
 
 def _sample_rows(lay, rng):
