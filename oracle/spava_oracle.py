@@ -39,6 +39,12 @@ Readings where the pages are silent (each also listed in the design notes):
   R6 lse is the natural log of the sum of exp(scale * q.k) over the row's keys.
   R7 the last block's passing set is never used (no later host), so it is not
      computed.
+  R8 selector variants ([PR] major comment 1, "What would settle it"): the
+     softmax form normalises each query-block row's logits over the block's
+     keys before summing; the context form sums the block's own causal
+     attention over its rows ("cumulative attention from all tokens in the
+     context block", read as attention within the block).  They change only
+     which keys pass; everything after the selection is as above.
 """
 from __future__ import annotations
 
@@ -160,6 +166,81 @@ def importance_scores(lay: Layout, Q, K, h: int) -> np.ndarray:
         logits = lay.scale * (q @ k.T)          # the Q_qr K^(h)T matrix
         out[kv] = logits.sum(axis=0)            # one importance per key
     return out
+
+
+# --------------------------------------------------------------------------
+# step 1, variants of the importance score.  The pages' selector is the
+# summed Q_qr K^(h)T above; the review ([PR] major comment 1, "What would
+# settle it") asks how its choice compares with others.  Two alternatives:
+#   softmax: each query-block row's attention over block h's keys (softmax of
+#            scale <q, k> over the block), summed per key over the rows and
+#            the KV head's query heads (the plain normalised form of R1);
+#   context: the review's oracle selector -- the cumulative attention each key
+#            of block h receives from all tokens of the block: every context
+#            row r of block h attends causally to the block's keys up to r
+#            (softmax over those keys), summed per key over the rows and the
+#            KV head's query heads.  Reading: "all tokens in the context block"
+#            attend within the block, i.e. the block's local causal attention.
+# --------------------------------------------------------------------------
+def _softmax_rows(z: np.ndarray) -> np.ndarray:
+    """Row-wise softmax of a logits matrix whose masked entries are -inf."""
+    m = z.max(axis=1, keepdims=True)
+    e = np.exp(z - m)
+    return e / e.sum(axis=1, keepdims=True)
+
+
+def importance_scores_softmax(lay: Layout, Q, K, h: int) -> np.ndarray:
+    """fp64 scores [Hkv, L_h]: sum over query-block rows i and query heads g
+    of the KV head of softmax_j(scale <q_ig, k_j>) over block h's keys."""
+    qs, s0, L = lay.query_start, lay.block_starts[h], lay.block_lens[h]
+    G, d = lay.group, lay.head_dim
+    out = np.empty((lay.num_kv_heads, L))
+    qrows = np.arange(qs, qs + lay.query_len)
+    for kv in range(lay.num_kv_heads):
+        q = np.stack([_take(Q, qrows, g) for g in range(kv * G, (kv + 1) * G)], axis=1).reshape(-1, d)
+        k = _take(K, np.arange(s0, s0 + L), kv)
+        out[kv] = _softmax_rows(lay.scale * (q @ k.T)).sum(axis=0)
+    return out
+
+
+def importance_scores_context(lay: Layout, Q, K, h: int) -> np.ndarray:
+    """fp64 scores [Hkv, L_h]: sum over block h's own rows r and the query
+    heads g of the KV head of the causal softmax, over the block's keys up to
+    r, of scale <q_rg, k_j>."""
+    s0, L = lay.block_starts[h], lay.block_lens[h]
+    G = lay.group
+    rows = np.arange(s0, s0 + L)
+    causal = np.arange(L)[None, :] <= np.arange(L)[:, None]      # key j visible to row r
+    out = np.zeros((lay.num_kv_heads, L))
+    for kv in range(lay.num_kv_heads):
+        k = _take(K, rows, kv)
+        for g in range(kv * G, (kv + 1) * G):
+            z = np.where(causal, lay.scale * (_take(Q, rows, g) @ k.T), -np.inf)
+            out[kv] += _softmax_rows(z).sum(axis=0)
+    return out
+
+
+SCORES = {"linear": importance_scores, "softmax": importance_scores_softmax,
+          "context": importance_scores_context}
+
+
+def compress_with(lay: Layout, Q, K, kind: str = "linear"):
+    """Scores and passing indices of blocks 0..V-2 under one of the selectors
+    (reading R7 for the last block, R2 for the selection)."""
+    scores = {h: SCORES[kind](lay, Q, K, h) for h in range(lay.V - 1)}
+    return scores, select_passing(lay, scores)
+
+
+def selection_overlap(lay: Layout, idx_a, idx_b) -> float:
+    """Fraction of the passing keys two selections share: sum over blocks and
+    KV heads of |A & B|, over the number of passing keys."""
+    both = total = 0
+    for h in range(lay.V - 1):
+        for kv in range(lay.num_kv_heads):
+            a, b = set(np.asarray(idx_a[h][kv]).tolist()), set(np.asarray(idx_b[h][kv]).tolist())
+            both += len(a & b)
+            total += len(a)
+    return both / total if total else 1.0
 
 
 # --------------------------------------------------------------------------

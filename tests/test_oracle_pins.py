@@ -372,3 +372,70 @@ def test_text_generator_needles_are_selected():
                     hits += p - lay.block_starts[h] in set(idx[h][kv].tolist())
                     total += 1
     assert total >= 40 and hits >= 0.75 * total, (hits, total)
+
+
+# ---------------------------------------------------------------- selector variants
+def test_softmax_scores_against_library_softmax():
+    """Per KV head, the softmax selector's score of key j is the sum over the
+    query block's rows and the KV head's query heads of torch.softmax over the
+    block's keys; the scores of a block sum to lq x G."""
+    lay, Q, K, Vv = _small(la=3, blocks=(20, 13, 17, 9), lq=7, lp=4)
+    for h in range(lay.V - 1):
+        s = oracle.importance_scores_softmax(lay, Q, K, h)
+        s0, L = lay.block_starts[h], lay.block_lens[h]
+        for kv in range(lay.num_kv_heads):
+            q = Q[lay.query_start:, kv * lay.group:(kv + 1) * lay.group]          # [lq, G, d]
+            z = torch.einsum("igc,jc->igj", q, K[s0:s0 + L, kv]) * lay.scale
+            want = torch.softmax(z, dim=-1).sum(dim=(0, 1)).numpy()
+            np.testing.assert_allclose(s[kv], want, rtol=1e-12, atol=1e-12)
+            assert abs(s[kv].sum() - lay.query_len * lay.group) < 1e-9
+
+
+def test_softmax_and_linear_agree_for_identical_queries():
+    """When every query-block query is the same vector, both selectors rank
+    keys by that vector's logit, so they keep the same keys."""
+    lay, Q, K, Vv = _small(lp=5)
+    Q[lay.query_start:] = Q[lay.query_start, 0]
+    _, lin = oracle.compress_with(lay, Q, K, "linear")
+    _, sm = oracle.compress_with(lay, Q, K, "softmax")
+    assert oracle.selection_overlap(lay, lin, sm) == 1.0
+
+
+def test_context_scores_against_library_causal_softmax():
+    """The context selector's score of key j is the sum over the block's own
+    rows (and the KV head's query heads) of torch.softmax over the causally
+    visible keys of the block, built here with an explicit mask."""
+    lay, Q, K, Vv = _small(la=4, blocks=(11, 8, 14, 6), lq=3, lp=3)
+    for h in range(lay.V - 1):
+        s = oracle.importance_scores_context(lay, Q, K, h)
+        s0, L = lay.block_starts[h], lay.block_lens[h]
+        mask = torch.triu(torch.ones(L, L, dtype=torch.bool), 1)      # key after row: hidden
+        for kv in range(lay.num_kv_heads):
+            want = torch.zeros(L, dtype=torch.float64)
+            for g in range(kv * lay.group, (kv + 1) * lay.group):
+                z = (Q[s0:s0 + L, g] @ K[s0:s0 + L, kv].T) * lay.scale
+                want += torch.softmax(z.masked_fill(mask, -math.inf), dim=-1).sum(dim=0)
+            np.testing.assert_allclose(s[kv], want.numpy(), rtol=1e-12, atol=1e-12)
+            assert abs(s[kv].sum() - L * lay.group) < 1e-9
+
+
+def test_context_scores_closed_form_for_equal_keys():
+    """All keys of a block equal: row r spreads its attention evenly over the
+    r + 1 keys it sees, so key j collects G x sum_{r >= j} 1 / (r + 1)."""
+    lay, Q, K, Vv = _small(la=2, blocks=(9, 5, 7, 4), lq=2, lp=2)
+    K[:] = torch.randn(lay.head_dim, dtype=torch.float64)
+    for h in range(lay.V - 1):
+        L = lay.block_lens[h]
+        want = lay.group * np.array([sum(1.0 / (r + 1) for r in range(j, L)) for j in range(L)])
+        s = oracle.importance_scores_context(lay, Q, K, h)
+        for kv in range(lay.num_kv_heads):
+            np.testing.assert_allclose(s[kv], want, rtol=1e-12)
+
+
+def test_selection_overlap_bounds():
+    lay, Q, K, Vv = _small(lp=4)
+    _, a = oracle.compress_with(lay, Q, K, "linear")
+    assert oracle.selection_overlap(lay, a, a) == 1.0
+    comp = {h: np.stack([np.setdiff1d(np.arange(lay.block_lens[h]), a[h][kv])[:lay.lp_eff(h)]
+                         for kv in range(lay.num_kv_heads)]) for h in a}
+    assert oracle.selection_overlap(lay, a, comp) == 0.0
