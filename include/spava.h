@@ -63,6 +63,15 @@ typedef enum {
 
 #define SPAVA_MAX_HOSTS 16   /* H; V = 2H <= 32 virtual hosts */
 
+/* Passing-key selectors (spava_problem_t.score_kind).  LINEAR is the pages'
+ * rule (Q_qr K^(h)T summed per key); the other two are the alternatives the
+ * review asks to compare it with ([PR] major comment 1, "What would settle
+ * it"); they change which keys pass, nothing else. */
+#define SPAVA_SCORE_LINEAR 0   /* sum over query-block rows of scale <q, k>              */
+#define SPAVA_SCORE_SOFTMAX 1  /* sum over query-block rows of softmax over the block    */
+#define SPAVA_SCORE_CONTEXT 2  /* sum over the block's own rows of their causal softmax
+                                  within the block (cumulative context attention)        */
+
 /* One layer's problem ([SC] Fig. 2 caption; [GN] Context Splitting;
  * [PR] ledger for la and lp). */
 typedef struct {
@@ -76,6 +85,7 @@ typedef struct {
   int32_t num_kv_heads;      /* Hkv >= 1, Hq % Hkv == 0                       */
   int32_t head_dim;          /* d in {64, 128}                                */
   float softmax_scale;       /* <= 0 selects 1/sqrt(d)                        */
+  int32_t score_kind;        /* SPAVA_SCORE_*; 0 = the pages' selector        */
 } spava_problem_t;
 
 /* Derived sizes, filled by spava_problem_sizes(). */
@@ -105,6 +115,18 @@ spava_status_t spava_workspace_size(const spava_problem_t* prob, size_t* bytes);
 spava_status_t spava_score(const spava_problem_t* prob, const void* Q,
                            const void* K, float* qsum, float* scores,
                            spava_stream_t stream);
+
+/* Step 1 under the selector prob->score_kind (any of SPAVA_SCORE_*), into
+ * `scores` (same layout as spava_score).  The two alternatives need two
+ * passes: the attention kernel computes every scoring row's log-normaliser
+ * over the block (softmax: the query block's rows over block h; context:
+ * block h's rows, causally over its own keys), then a tensor-core kernel
+ * sums exp(scale <q, k> - lse) per key.  `workspace` (>= spava_workspace_size
+ * bytes for this problem, 256-byte aligned) holds the first pass's output.
+ * spava_score itself returns SPAVA_ERR_UNSUPPORTED for these selectors. */
+spava_status_t spava_score_variant(const spava_problem_t* prob, const void* Q,
+                                   const void* K, float* scores, void* workspace,
+                                   size_t ws_bytes, spava_stream_t stream);
 
 /* Step 2, top-lp per block and KV head ([PR] "What carries the argument":
  * each context block compressed to its top-lp key-value pairs).  Larger
@@ -165,7 +187,8 @@ spava_status_t spava_lse_merge(const spava_problem_t* prob, const float* O_part,
  * for it only before reading the passing buffer.  The work list is checked
  * before anything is launched (SPAVA_ERR_UNSUPPORTED: more than 6144 work
  * items of two 128-row tiles).  Blocks longer than 24576 keys fall back to
- * the three stage kernels of steps 1-3. */
+ * the three stage kernels of steps 1-3, and so do the selectors other than
+ * SPAVA_SCORE_LINEAR (spava_score_variant, top-lp, gather). */
 spava_status_t spava_layer_fwd(const spava_problem_t* prob, const void* Q,
                                const void* K, const void* V, void* O,
                                float* lse, void* workspace, size_t ws_bytes,

@@ -44,6 +44,7 @@ struct Region {
 
 struct Plan {
   int H = 0, V = 0, la = 0, lq = 0, lp = 0, Hq = 0, Hkv = 0, d = 0, G = 0;
+  int score_kind = 0;   // SPAVA_SCORE_*
   float scale = 0.f;
   int64_t n = 0, qs = 0, score_cols = 0, passing_rows = 0;
   int32_t L[kMaxV] = {}, start[kMaxV] = {}, lpe[kMaxV] = {}, poff[kMaxV + 1] = {};
@@ -55,7 +56,7 @@ struct Plan {
   int n_merge = 0;   // merge counters: one per (pair of 128-row query tiles, query head)
   // workspace carving (bytes from the workspace base)
   size_t ws_qsum = 0, ws_scores = 0, ws_idx = 0, ws_kp = 0, ws_vp = 0, ws_opart = 0,
-         ws_lsepart = 0, ws_count = 0, ws_total = 0;
+         ws_lsepart = 0, ws_count = 0, ws_vo = 0, ws_vlse = 0, ws_total = 0;
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -92,6 +93,7 @@ inline spava_status_t make_plan(const spava_problem_t* p, Plan* pl) {
   if (p->num_q_heads % p->num_kv_heads) return SPAVA_ERR_INVALID_ARG;
   if (p->head_dim != 64 && p->head_dim != 128) return SPAVA_ERR_UNSUPPORTED;
   if (!(p->softmax_scale == p->softmax_scale)) return SPAVA_ERR_INVALID_ARG;  // NaN
+  if (p->score_kind < SPAVA_SCORE_LINEAR || p->score_kind > SPAVA_SCORE_CONTEXT) return SPAVA_ERR_INVALID_ARG;
   Plan& P = *pl;
   P = Plan();
   P.H = p->num_hosts;
@@ -103,6 +105,7 @@ inline spava_status_t make_plan(const spava_problem_t* p, Plan* pl) {
   P.Hkv = p->num_kv_heads;
   P.d = p->head_dim;
   P.G = P.Hq / P.Hkv;
+  P.score_kind = p->score_kind;
   P.scale = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / std::sqrt(static_cast<float>(P.d));
   int64_t pos = P.la;
   for (int h = 0; h < P.V; ++h) {
@@ -185,8 +188,37 @@ inline spava_status_t make_plan(const spava_problem_t* p, Plan* pl) {
   P.ws_lsepart = carve(sizeof(float) * static_cast<size_t>(P.V) * P.Hq * P.lq);
   P.n_merge = ((P.lq + 2 * kBM - 1) / (2 * kBM)) * P.Hq;
   P.ws_count = carve(sizeof(int32_t) * static_cast<size_t>(P.n_merge));
+  if (P.score_kind == SPAVA_SCORE_CONTEXT) {   // first pass of the context selector: O and lse of the block rows
+    P.ws_vo = carve(2ull * static_cast<size_t>(P.n) * P.Hq * P.d);
+    P.ws_vlse = carve(sizeof(float) * static_cast<size_t>(P.Hq) * P.n);
+  }
   P.ws_total = off;
   return SPAVA_OK;
+}
+
+// The first pass of a selector variant as attention regions over the blocks
+// h < V-1: softmax -> the query block's rows over block h's keys (written as
+// host h's query partial); context -> block h's rows causally over its own
+// keys (written as rows).  Replaces the plan's regions, tiles and items.
+inline void make_variant_regions(Plan* pl) {
+  Plan& P = *pl;
+  P.nregions = 0;
+  P.tiles = 0;
+  P.items = 0;
+  P.passing_rows = 0;   // no region reads the passing buffer
+  for (int h = 0; h < P.V - 1; ++h) {
+    Region& R = P.regions[P.nregions++];
+    const bool ctx = P.score_kind == SPAVA_SCORE_CONTEXT;
+    R.row_start = ctx ? P.start[h] : static_cast<int32_t>(P.qs);
+    R.nrows = ctx ? P.L[h] : P.lq;
+    R.out_kind = ctx ? kOutRows : kOutPartial;
+    R.host = h;
+    R.nseg = 1;
+    R.seg[0] = Seg{kSrcMain, P.start[h], P.L[h], ctx ? 1 : 0};
+    const int nt = (R.nrows + kBM - 1) / kBM;
+    P.tiles += nt;
+    P.items += (nt + 1) / 2;
+  }
 }
 
 // Cost-ordered work items: (region << 20) | pair, one CTA per pair of

@@ -14,6 +14,7 @@
 #include "compress.cuh"
 #include "compress_fused.cuh"
 #include "merge.cuh"
+#include "score_variants.cuh"
 #include "plan.hpp"
 #include "ptx.cuh"
 
@@ -101,6 +102,12 @@ spava_status_t device_setup(const DeviceSetup** out) {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0) s.sm_count = n;
     spava_status_t st = setup_attn<128>();
     if (st == SPAVA_OK) st = setup_attn<64>();
+    if (st == SPAVA_OK &&
+        (cudaFuncSetAttribute(colsum_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              ColsumCfg<128>::kSmemBytes) != cudaSuccess ||
+         cudaFuncSetAttribute(colsum_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              ColsumCfg<64>::kSmemBytes) != cudaSuccess))
+      st = SPAVA_ERR_CUDA;
     const int csmem = compress_smem_bytes(kCompressMaxBlock);
     if (st == SPAVA_OK &&
         (cudaFuncSetAttribute(compress_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, csmem) !=
@@ -128,6 +135,7 @@ int sm_count() {
 // skip the sort and the encoding.
 struct AttnKey {
   int device;
+  int tag;   // which regions: 0 the layer's, else the first pass of selector `tag`
   int32_t H, la, lq, lp, Hq, Hkv, d;
   float scale;
   int32_t L[kMaxV];
@@ -147,11 +155,12 @@ std::mutex g_attn_mu;
 AttnEntry g_attn_cache[kAttnCacheSize];
 uint64_t g_attn_clock = 0;
 
-AttnKey attn_key(const Plan& P, int dev, const void* Q, const void* K, const void* V, const void* Kp,
-                 const void* Vp) {
+AttnKey attn_key(const Plan& P, int dev, int tag, const void* Q, const void* K, const void* V,
+                 const void* Kp, const void* Vp) {
   AttnKey k;
   std::memset(&k, 0, sizeof(k));   // padding included, for the byte-wise compare
   k.device = dev;
+  k.tag = tag;
   k.H = P.H;
   k.la = P.la;
   k.lq = P.lq;
@@ -207,11 +216,11 @@ spava_status_t build_attn(const Plan& P, const void* Q, const void* K, const voi
 
 // The cached parameter block for these inputs, built on a miss.  The caller
 // holds g_attn_mu while it uses the returned entry.
-spava_status_t attn_entry(const Plan& P, const void* Q, const void* K, const void* V, const void* Kp,
-                          const void* Vp, AttnEntry** out) {
+spava_status_t attn_entry(const Plan& P, int tag, const void* Q, const void* K, const void* V,
+                          const void* Kp, const void* Vp, AttnEntry** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return SPAVA_ERR_CUDA;
-  const AttnKey key = attn_key(P, dev, Q, K, V, Kp, Vp);
+  const AttnKey key = attn_key(P, dev, tag, Q, K, V, Kp, Vp);
   AttnEntry* victim = &g_attn_cache[0];
   for (AttnEntry& e : g_attn_cache) {
     if (e.prm && e.key == key) {
@@ -379,7 +388,7 @@ spava_status_t run_compress(const Plan& P, const void* Q, const void* K, const v
 // counters.
 spava_status_t run_attn(const Plan& P, const void* Q, const void* K, const void* V, const void* Kp,
                         const void* Vp, void* O, float* lse, float* O_part, float* lse_part,
-                        int32_t* merge_count, bool dependent, cudaStream_t st) {
+                        int32_t* merge_count, bool dependent, cudaStream_t st, int tag = 0) {
   if (!Q || !K || !V || !O || !lse || !O_part || !lse_part) return SPAVA_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(O_part))
     return SPAVA_ERR_INVALID_ARG;
@@ -390,7 +399,7 @@ spava_status_t run_attn(const Plan& P, const void* Q, const void* K, const void*
   if (s != SPAVA_OK) return s;
   std::lock_guard<std::mutex> lock(g_attn_mu);
   AttnEntry* e = nullptr;
-  if ((s = attn_entry(P, Q, K, V, Kp, Vp, &e)) != SPAVA_OK) return s;
+  if ((s = attn_entry(P, tag, Q, K, V, Kp, Vp, &e)) != SPAVA_OK) return s;
   AttnParams& prm = *e->prm;
   prm.O = static_cast<__nv_bfloat16*>(O);
   prm.lse = lse;
@@ -433,6 +442,58 @@ spava_status_t run_merge(const Plan& P, const float* O_part, const float* lse_pa
   return last_launch();
 }
 
+// Step 1 under a selector variant (P.score_kind != linear), two passes:
+// the attention kernel on the variant's regions gives every scoring row's
+// lse over the block (softmax: into the query-partial slots; context: into
+// the workspace's row outputs), then colsum_kernel sums the probabilities
+// per key.  `ws` is the layer's workspace.
+spava_status_t run_score_variant(const Plan& P, const void* Q, const void* K, float* scores, uint8_t* ws,
+                                 cudaStream_t st) {
+  if (!Q || !K || !scores || !aligned16(Q) || !aligned16(K)) return SPAVA_ERR_INVALID_ARG;
+  if (P.V < 2 || P.score_cols == 0) return SPAVA_OK;
+  Plan PV = P;
+  make_variant_regions(&PV);
+  if (PV.items > kMaxItems) return SPAVA_ERR_UNSUPPORTED;
+  const bool ctx = P.score_kind == kScoreContext;
+  float* O_part = reinterpret_cast<float*>(ws + P.ws_opart);
+  float* lse_part = reinterpret_cast<float*>(ws + P.ws_lsepart);
+  void* vo = ctx ? static_cast<void*>(ws + P.ws_vo) : static_cast<void*>(O_part);
+  float* vlse = ctx ? reinterpret_cast<float*>(ws + P.ws_vlse) : lse_part;
+  spava_status_t s = run_attn(PV, Q, K, K, nullptr, nullptr, vo, vlse, O_part, lse_part, nullptr, false, st,
+                              P.score_kind);
+  if (s != SPAVA_OK) return s;
+  auto prm = std::make_unique<ColsumParams>();
+  std::memset(prm.get(), 0, sizeof(ColsumParams));
+  if (!make_tmap(&prm->tm_q, Q, P.d, P.Hq, P.n) || !make_tmap(&prm->tm_k, K, P.d, P.Hkv, P.n)) return SPAVA_ERR_CUDA;
+  prm->scores = scores;
+  prm->lse = ctx ? vlse : lse_part;
+  prm->kind = P.score_kind;
+  prm->Hq = P.Hq;
+  prm->G = P.G;
+  prm->lq = P.lq;
+  prm->qs = static_cast<int32_t>(P.qs);
+  prm->n = static_cast<int32_t>(P.n);
+  prm->la = P.la;
+  prm->V = P.V;
+  prm->score_cols = P.score_cols;
+  prm->scale_log2 = P.scale * 1.44269504088896340736f;
+  prm->nblocks = P.V - 1;
+  int tiles = 0;
+  for (int h = 0; h < P.V - 1; ++h) {
+    prm->start[h] = P.start[h];
+    prm->L[h] = P.L[h];
+    prm->tile0[h] = tiles;
+    tiles += (P.L[h] + 127) / 128;
+  }
+  prm->tile0[P.V - 1] = tiles;
+  const dim3 grid(static_cast<unsigned>(tiles), static_cast<unsigned>(P.Hkv));
+  if (P.d == 128)
+    colsum_kernel<128><<<grid, ColsumCfg<128>::kThreads, ColsumCfg<128>::kSmemBytes, st>>>(*prm);
+  else
+    colsum_kernel<64><<<grid, ColsumCfg<64>::kThreads, ColsumCfg<64>::kSmemBytes, st>>>(*prm);
+  return last_launch();
+}
+
 // The whole layer with its intermediates carved from `ws` (P.ws_total bytes,
 // 256-byte aligned): compression (one launch, or the three stage kernels for
 // blocks too long for it), then attention with the query-partial merge in
@@ -455,10 +516,16 @@ spava_status_t run_layer(const Plan& P, uint8_t* ws, const void* Q, const void* 
     if ((s = device_setup(&ds)) != SPAVA_OK) return s;
     std::lock_guard<std::mutex> lock(g_attn_mu);
     AttnEntry* e = nullptr;
-    if ((s = attn_entry(P, Q, K, V, Kp, Vp, &e)) != SPAVA_OK) return s;
+    if ((s = attn_entry(P, 0, Q, K, V, Kp, Vp, &e)) != SPAVA_OK) return s;
   }
   bool dependent = false;
-  if (P.lp > 0 && compress_fits(P)) {   // steps 1-3 in one launch; it also zeroes the merge counters
+  if (P.lp > 0 && P.score_kind != kScoreLinear) {   // a selector variant: two scoring passes, top-lp, gather
+    if ((s = run_score_variant(P, Q, K, scores, ws, st)) != SPAVA_OK) return s;
+    if ((s = run_topk(P, scores, idx, st)) != SPAVA_OK) return s;
+    if ((s = run_gather(P, K, V, idx, Kp, Vp, st)) != SPAVA_OK) return s;
+    if (cudaMemsetAsync(count, 0, sizeof(int32_t) * static_cast<size_t>(P.n_merge), st) != cudaSuccess)
+      return SPAVA_ERR_CUDA;
+  } else if (P.lp > 0 && compress_fits(P)) {   // steps 1-3 in one launch; it also zeroes the merge counters
     if ((s = run_compress(P, Q, K, V, qsum, scores, idx, Kp, Vp, count, st)) != SPAVA_OK) return s;
     dependent = true;
   } else {
@@ -520,7 +587,24 @@ spava_status_t spava_score(const spava_problem_t* prob, const void* Q, const voi
   Plan P;
   spava_status_t s = make_plan(prob, &P);
   if (s != SPAVA_OK) return s;
+  if (P.score_kind != kScoreLinear) return SPAVA_ERR_UNSUPPORTED;   // spava_score_variant
   return run_score(P, Q, K, qsum, scores, reinterpret_cast<cudaStream_t>(stream));
+}
+
+spava_status_t spava_score_variant(const spava_problem_t* prob, const void* Q, const void* K, float* scores,
+                                   void* workspace, size_t ws_bytes, spava_stream_t stream) {
+  Plan P;
+  spava_status_t s = make_plan(prob, &P);
+  if (s != SPAVA_OK) return s;
+  if (P.score_kind == kScoreLinear) {   // the pages' selector needs no workspace
+    if (!workspace || ws_bytes < P.ws_total) return SPAVA_ERR_WORKSPACE;
+    float* qsum = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + P.ws_qsum);
+    return run_score(P, Q, K, qsum, scores, reinterpret_cast<cudaStream_t>(stream));
+  }
+  if (!workspace || ws_bytes < P.ws_total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return SPAVA_ERR_WORKSPACE;
+  return run_score_variant(P, Q, K, scores, static_cast<uint8_t*>(workspace),
+                           reinterpret_cast<cudaStream_t>(stream));
 }
 
 spava_status_t spava_select_topk(const spava_problem_t* prob, const float* scores, int32_t* idx,

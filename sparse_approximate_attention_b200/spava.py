@@ -16,6 +16,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libspava.so")
 
+SCORE_KINDS = {"linear": 0, "softmax": 1, "context": 2}   # SPAVA_SCORE_*
 STATUS = {0: "SPAVA_OK", 1: "SPAVA_ERR_INVALID_ARG", 2: "SPAVA_ERR_UNSUPPORTED",
           3: "SPAVA_ERR_WORKSPACE", 4: "SPAVA_ERR_CUDA", 5: "SPAVA_ERR_DEVICE"}
 
@@ -31,7 +32,7 @@ class _Problem(ctypes.Structure):
                 ("block_lens", ctypes.POINTER(ctypes.c_int32)), ("query_len", ctypes.c_int32),
                 ("lp", ctypes.c_int32), ("num_q_heads", ctypes.c_int32),
                 ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
-                ("softmax_scale", ctypes.c_float)]
+                ("softmax_scale", ctypes.c_float), ("score_kind", ctypes.c_int32)]
 
 
 class _Sizes(ctypes.Structure):
@@ -48,6 +49,7 @@ _SIGS = {
     "spava_problem_sizes": [_PP, ctypes.POINTER(_Sizes)],
     "spava_workspace_size": [_PP, ctypes.POINTER(ctypes.c_size_t)],
     "spava_score": [_PP, _VP, _VP, _VP, _VP, _VP],
+    "spava_score_variant": [_PP, _VP, _VP, _VP, _VP, ctypes.c_size_t, _VP],
     "spava_select_topk": [_PP, _VP, _VP, _VP],
     "spava_gather_passing": [_PP, _VP, _VP, _VP, _VP, _VP, _VP],
     "spava_compress": [_PP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
@@ -90,20 +92,22 @@ class Problem:
 
     def __init__(self, num_hosts: int, anchor_len: int, block_lens: Sequence[int],
                  query_len: int, lp: int, num_q_heads: int, num_kv_heads: int,
-                 head_dim: int, softmax_scale: float = 0.0):
+                 head_dim: int, softmax_scale: float = 0.0, score_kind: str = "linear"):
         self.num_hosts, self.anchor_len = int(num_hosts), int(anchor_len)
         self.block_lens = [int(x) for x in block_lens]
         self.query_len, self.lp = int(query_len), int(lp)
         self.num_q_heads, self.num_kv_heads = int(num_q_heads), int(num_kv_heads)
         self.head_dim, self.softmax_scale = int(head_dim), float(softmax_scale)
+        self.score_kind = score_kind
         self._arr = (ctypes.c_int32 * max(1, len(self.block_lens)))(*self.block_lens)
         self._c = _Problem(self.num_hosts, self.anchor_len, self._arr, self.query_len, self.lp,
-                           self.num_q_heads, self.num_kv_heads, self.head_dim, self.softmax_scale)
+                           self.num_q_heads, self.num_kv_heads, self.head_dim, self.softmax_scale,
+                           SCORE_KINDS[score_kind])
 
     @classmethod
-    def from_workload(cls, wl) -> "Problem":
+    def from_workload(cls, wl, score_kind: str = "linear") -> "Problem":
         return cls(wl.num_hosts, wl.anchor_len, wl.block_lens, wl.query_len, wl.lp,
-                   wl.num_q_heads, wl.num_kv_heads, wl.head_dim)
+                   wl.num_q_heads, wl.num_kv_heads, wl.head_dim, score_kind=score_kind)
 
     @property
     def ref(self):
@@ -154,6 +158,21 @@ def score(p: Problem, Q, K, qsum=None, scores=None, stream=None):
     _need(scores, torch.float32, sh["scores"], "scores")
     _check("spava_score", lib().spava_score(p.ref, _ptr(Q), _ptr(K), _ptr(qsum), _ptr(scores), _stream(stream)))
     return qsum, scores
+
+
+def score_variant(p: Problem, Q, K, scores=None, workspace=None, stream=None):
+    """Step 1 under the problem's selector (p.score_kind), into scores [Hkv, S]."""
+    sz, sh = _shapes(p)
+    _need(Q, torch.bfloat16, sh["Q"], "Q")
+    _need(K, torch.bfloat16, sh["K"], "K")
+    scores = torch.empty(sh["scores"], dtype=torch.float32, device=Q.device) if scores is None else scores
+    _need(scores, torch.float32, sh["scores"], "scores")
+    if workspace is None:
+        workspace = torch.empty(max(1, sz["workspace_bytes"]), dtype=torch.uint8, device=Q.device)
+    _check("spava_score_variant", lib().spava_score_variant(
+        p.ref, _ptr(Q), _ptr(K), _ptr(scores), _ptr(workspace),
+        ctypes.c_size_t(workspace.numel() * workspace.element_size()), _stream(stream)))
+    return scores
 
 
 def select_topk(p: Problem, scores, idx=None, stream=None):
