@@ -19,7 +19,8 @@
 // other two with setmaxnreg):
 //   warp 0     TMA producer: Q0 and Q1 once, then K and V tiles into separate
 //              rings (K runs one tile ahead of V, the order the MMAs use them)
-//   warp 1     TMEM owner and single-thread MMA issuer.  Per key tile j:
+//   warp 1     TMEM owner and MMA issuer (warp-wide loop, one elected lane
+//              issues).  Per key tile j:
 //              S0 = Q0 K_j^T, O1 += P1 V_{j-1}, S1 = Q1 K_j^T, O0 += P0 V_j,
 //              so the tensor pipe works on one tile while the other tile's
 //              softmax runs
@@ -291,7 +292,10 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // The whole warp runs this loop; elect.sync picks the lane that issues
+    // each MMA and commit (ptx.cuh: mma_*_warp), and the waits are taken by
+    // every lane and voted, so control flow stays warp-uniform.
+    {
       constexpr uint32_t kIdescQK = idesc_bf16_f32(128, kBN, false, false);
       constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, false, true);
       // Descriptor high words are constant (SBO 1024 B, version 1, 128-B
@@ -302,6 +306,9 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1)
       const uint32_t q_lo = (sQ >> 4) | (1u << 16);
       const uint32_t k_lo = (sK >> 4) | (1u << 16);
       const uint32_t v_lo = (sV >> 4) | ((static_cast<uint32_t>(C::kSlabBytes) >> 4) << 16);
+      auto wait = [&](uint32_t bar, uint32_t parity) {
+        return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+      };
       // S_t = Q_t K_j^T into TMEM buffer t
       auto issue_s = [&](int t, int j) {
         const uint32_t tS = tmem + 256u + 128u * t;
@@ -310,11 +317,10 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1)
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const uint32_t off = ((k >> 2) * C::kSlabBytes + (k & 3) * 32) >> 4;
-          mma_ss(tS, desc(qa + off), desc(kb + off), kIdescQK, k > 0 ? 1u : 0u);
+          mma_ss_warp(tS, desc(qa + off), desc(kb + off), kIdescQK, k > 0 ? 1u : 0u);
         }
-        mma_commit(BAR_SF(t));
+        mma_commit_warp(BAR_SF(t));
       };
-      // O_t += P_t V_j once P_t (softmax of tile t) and V_j are ready
       // O_t += P_t V_j once P_t (softmax of tile t) is ready; V_j's arrival
       // is awaited by the caller beforehand, off the P-ready path.
       auto issue_pv = [&](int t, int j, bool release_v, bool last) -> bool {
@@ -326,20 +332,19 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1)
         // the softmax still computes the second half
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-          if (!mbar_wait(BAR_PF(t, half), j & 1, abort_flag)) return false;
+          if (!wait(BAR_PF(t, half), j & 1)) return false;
           tc_fence_after();
 #pragma unroll
           for (int k = 4 * half; k < 4 * half + 4; ++k)
-            mma_ts(tO, tP + k * 8, desc(vb + ((k * 2048) >> 4)), kIdescPV, (j > 0 || k > 0) ? 1u : 0u);
+            mma_ts_warp(tO, tP + k * 8, desc(vb + ((k * 2048) >> 4)), kIdescPV, (j > 0 || k > 0) ? 1u : 0u);
         }
-        if (last) mma_commit(BAR_OD(t));   // single phase: O_t is final
-        if (release_v) mma_commit(BAR_VE(st));
+        if (last) mma_commit_warp(BAR_OD(t));   // single phase: O_t is final
+        if (release_v) mma_commit_warp(BAR_VE(st));
         return true;
       };
-      auto wait_v = [&](int j) { return mbar_wait(BAR_VF(j % VS), (j / VS) & 1, abort_flag); };
-      bool ok = mbar_wait(BAR_Q, 0, abort_flag);
+      bool ok = wait(BAR_Q, 0);
       for (int j = 0; ok && j < ntk; ++j) {
-        ok = mbar_wait(BAR_KF(j % KS), (j / KS) & 1, abort_flag);
+        ok = wait(BAR_KF(j % KS), (j / KS) & 1);
         if (!ok) break;
         tc_fence_after();
         if (j < nt0) issue_s(0, j);
@@ -348,8 +353,8 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1)
           if (!ok) break;
         }
         if (j < nt1) issue_s(1, j);
-        mma_commit(BAR_KE(j % KS));
-        ok = wait_v(j);                    // V_j is needed by O0 (now) or O1 (next)
+        mma_commit_warp(BAR_KE(j % KS));
+        ok = wait(BAR_VF(j % VS), (j / VS) & 1);   // V_j is needed by O0 (now) or O1 (next)
         if (!ok) break;
         if (j < nt0) {
           ok = issue_pv(0, j, j >= nt1, j == nt0 - 1);   // V_j is Q0's alone when Q1 does not read it
@@ -357,7 +362,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1)
         }
       }
       if (ok && nt1 > 0) issue_pv(1, nt1 - 1, true, true);
-      mma_commit(BAR_FIN);   // every MMA issued above has finished once this lands
+      mma_commit_warp(BAR_FIN);   // every MMA issued above has finished once this lands
       mbar_wait_drain(BAR_FIN, 0);
     }
   } else if (warp >= 4) {
@@ -376,6 +381,17 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1)
     float m = -INFINITY;   // running max of the scaled logits, log2 units
     float l = 0.f;
     bool ok = true;
+    // Keys of each segment this row sees, computed once (the loop below then
+    // reads no segment descriptors from parameter memory).
+    int seg_lim[kMaxSegs];
+#pragma unroll
+    for (int s = 0; s < kMaxSegs; ++s) {
+      seg_lim[s] = 0;
+      if (s < nseg) {
+        const Seg& sg = R.seg[s];
+        seg_lim[s] = sg.causal ? min(sg.len, row - sg.start + 1) : sg.len;
+      }
+    }
     TileIter it = iter_begin();
     for (int j = 0; j < nt; ++j) {
       ok = __all_sync(0xffffffffu, mbar_wait(BAR_SF(qt), j & 1, abort_flag));
@@ -391,9 +407,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1)
           x[c * 16 + e] = make_float2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]));
       }
       tmem_wait_ld();
-      const Seg& sg = R.seg[it.s];
-      int lim = sg.len;
-      if (sg.causal) lim = min(lim, row - sg.start + 1);
+      const int lim = it.s == 0 ? seg_lim[0] : it.s == 1 ? seg_lim[1] : seg_lim[2];
       const int nvalid = lim - it.kt * kBN;
       if (nvalid < kBN) {
 #pragma unroll
