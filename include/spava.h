@@ -86,9 +86,30 @@ typedef struct {
   int32_t head_dim;          /* d in {64, 128}                                */
   float softmax_scale;       /* <= 0 selects 1/sqrt(d)                        */
   int32_t score_kind;        /* SPAVA_SCORE_*; 0 = the pages' selector        */
+  uint32_t host_mask;        /* 0 = every virtual host (the whole layer on one
+                                GPU).  Otherwise the virtual hosts this caller
+                                computes, bit h for host h (bits >= V must be
+                                0): the compression of block h (h < V-1), the
+                                context rows of block h and host h's query
+                                partial; the anchor rows go with bit 0.  This
+                                is the pages' own split of the 2H virtual
+                                hosts over GPUs ([SC] Fig. 2 and Fig. 4
+                                captions: GPU p holds hosts p and 2H-1-p; [PR]
+                                "What carries the argument": the passing
+                                blocks are all-gathered across hosts): each
+                                GPU runs spava_compress and spava_attn_fwd
+                                with its mask, the caller exchanges the Kp/Vp
+                                rows and the query partials between the GPUs,
+                                and spava_lse_merge merges all V partials.
+                                spava_compress, spava_attn_fwd,
+                                spava_problem_sizes and spava_lse_merge
+                                accept a partial mask (lse_merge always merges
+                                all V partials); every other call returns
+                                SPAVA_ERR_UNSUPPORTED for it.                 */
 } spava_problem_t;
 
-/* Derived sizes, filled by spava_problem_sizes(). */
+/* Derived sizes, filled by spava_problem_sizes().  attn_pairs, attn_flops and
+ * attn_tiles count the rows host_mask selects. */
 typedef struct {
   int64_t seq_len;        /* n                                               */
   int64_t query_start;    /* la + sum L_h                                     */
@@ -150,7 +171,9 @@ spava_status_t spava_gather_passing(const spava_problem_t* prob, const void* K,
  * (block, KV head) streams K^(h) once, selects in shared memory and copies the
  * kept rows.  Every block length must be <= 24576 (SPAVA_ERR_UNSUPPORTED
  * otherwise; the separate stage calls have no such limit).  With lp = 0 it
- * does nothing. */
+ * does nothing.  With a partial host_mask only the selected blocks are
+ * compressed: their scores, idx and Kp/Vp rows (at their offsets off_h of the
+ * full buffer) are written, nothing else. */
 spava_status_t spava_compress(const spava_problem_t* prob, const void* Q,
                               const void* K, const void* V, float* qsum,
                               float* scores, int32_t* idx, void* Kp, void* Vp,
@@ -162,7 +185,10 @@ spava_status_t spava_compress(const spava_problem_t* prob, const void* Q,
  *   anchor rows r < la: keys 0..r;
  *   context rows of host h: A, Kp rows [0, off_h), and B^(h) keys up to r;
  *   query rows, partial of host h: B^(h) (host 0 also A and B_qr up to r).
- * Writes O / lse for anchor and context rows, and O_part / lse_part. */
+ * Writes O / lse for anchor and context rows, and O_part / lse_part.  With a
+ * partial host_mask only the selected hosts' rows and partials are written
+ * (context rows of host h still read Kp rows [0, off_h), which the caller must
+ * have filled with the other hosts' passing rows). */
 spava_status_t spava_attn_fwd(const spava_problem_t* prob, const void* Q,
                               const void* K, const void* V, const void* Kp,
                               const void* Vp, void* O, float* lse,

@@ -6,7 +6,8 @@
 // review), "What carries the argument": each context block is compressed to
 // its top-lp key-value pairs ranked by Q_qr K^T and gathered by later hosts.
 //
-// One thread-block cluster of kCompressCtas CTAs per (block h < V-1, KV head),
+// One thread-block cluster of kCompressCtas CTAs per (block h < V-1, KV head)
+// (all such blocks, or those a host mask selects),
 // for blocks of up to kCompressMaxBlock keys:
 //   1. each CTA sums a slice of the query block's (row, head) pairs of the KV
 //      group; the slices are added in rank order through distributed shared
@@ -59,6 +60,7 @@ struct CompressParams {
   // no separate launch is needed); null when called on its own
   int32_t* merge_count;
   int32_t n_merge;
+  int32_t blk[kMaxV];     // the compressed blocks, one per grid row (all h < V-1, or a host mask's)
 };
 
 template <int D>
@@ -86,12 +88,12 @@ __global__ void __cluster_dims__(kCompressCtas, 1, 1) __launch_bounds__(kCompres
 
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = static_cast<int>(cluster.block_rank());
-  const int h = blockIdx.y, kv = blockIdx.z;
+  const int h = p.blk[blockIdx.y], kv = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // The attention launch that follows may start on the SMs this grid leaves
   // free; it reads nothing written here before its griddepcontrol.wait.
   if (tid == 0) grid_dependents_launch();
-  if (p.merge_count != nullptr && blockIdx.x == 0 && h == 0 && kv == 0)
+  if (p.merge_count != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && kv == 0)
     for (int i = tid; i < p.n_merge; i += kCompressThreads) p.merge_count[i] = 0;
   const int L = p.L[h], kk = p.k[h];
   const int j0 = static_cast<int>((static_cast<int64_t>(L) * rank) / kCompressCtas);

@@ -45,6 +45,10 @@ struct Region {
 struct Plan {
   int H = 0, V = 0, la = 0, lq = 0, lp = 0, Hq = 0, Hkv = 0, d = 0, G = 0;
   int score_kind = 0;   // SPAVA_SCORE_*
+  uint64_t hmask = 0;   // selected virtual hosts (all V bits when the problem's mask is 0)
+  bool partial = false; // some virtual host is not selected
+  int ncblk = 0;        // selected compressed blocks (h < V-1)
+  int32_t cblk[kMaxV] = {};
   float scale = 0.f;
   int64_t n = 0, qs = 0, score_cols = 0, passing_rows = 0;
   int32_t L[kMaxV] = {}, start[kMaxV] = {}, lpe[kMaxV] = {}, poff[kMaxV + 1] = {};
@@ -107,6 +111,13 @@ inline spava_status_t make_plan(const spava_problem_t* p, Plan* pl) {
   P.G = P.Hq / P.Hkv;
   P.score_kind = p->score_kind;
   P.scale = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / std::sqrt(static_cast<float>(P.d));
+  const uint64_t all = (uint64_t(1) << P.V) - 1;
+  if (static_cast<uint64_t>(p->host_mask) & ~all) return SPAVA_ERR_INVALID_ARG;
+  P.hmask = p->host_mask ? static_cast<uint64_t>(p->host_mask) : all;
+  P.partial = P.hmask != all;
+  auto sel = [&](int h) { return ((P.hmask >> h) & 1u) != 0; };
+  for (int h = 0; h < P.V - 1; ++h)
+    if (sel(h)) P.cblk[P.ncblk++] = h;
   int64_t pos = P.la;
   for (int h = 0; h < P.V; ++h) {
     int32_t L = p->block_lens[h];
@@ -142,6 +153,7 @@ inline spava_status_t make_plan(const spava_problem_t* p, Plan* pl) {
     R.seg[R.nseg++] = Seg{src, s, len, causal};
   };
   for (int h = 0; h < P.V; ++h) {   // query rows, partial of host h
+    if (!sel(h)) continue;
     Region& R = add(static_cast<int32_t>(P.qs), P.lq, kOutPartial, h);
     if (h == 0) {
       seg(R, kSrcMain, 0, P.la + P.L[0], 0);       // A and B^(0), contiguous
@@ -152,6 +164,7 @@ inline spava_status_t make_plan(const spava_problem_t* p, Plan* pl) {
   }
   for (int i = 0; i < P.V; ++i) {   // context rows, ZigZag order 0, V-1, 1, V-2, ...
     int h = (i % 2 == 0) ? i / 2 : P.V - 1 - i / 2;
+    if (!sel(h)) continue;
     Region& R = add(P.start[h], P.L[h], kOutRows, h);
     if (h == 0) {
       seg(R, kSrcMain, 0, P.la + P.L[0], 1);       // A then causal B^(0): plain causal
@@ -161,7 +174,7 @@ inline spava_status_t make_plan(const spava_problem_t* p, Plan* pl) {
       seg(R, kSrcMain, P.start[h], P.L[h], 1);
     }
   }
-  if (P.la > 0) {
+  if (P.la > 0 && sel(0)) {   // the anchor rows go with virtual host 0
     Region& R = add(0, P.la, kOutRows, -1);
     seg(R, kSrcMain, 0, P.la, 1);
   }

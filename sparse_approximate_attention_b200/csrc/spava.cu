@@ -138,6 +138,7 @@ struct AttnKey {
   int tag;   // which regions: 0 the layer's, else the first pass of selector `tag`
   int32_t H, la, lq, lp, Hq, Hkv, d;
   float scale;
+  uint64_t hmask;
   int32_t L[kMaxV];
   const void *Q, *K, *V, *Kp, *Vp;
   bool operator==(const AttnKey& o) const { return std::memcmp(this, &o, sizeof(AttnKey)) == 0; }
@@ -169,6 +170,7 @@ AttnKey attn_key(const Plan& P, int dev, int tag, const void* Q, const void* K, 
   k.Hkv = P.Hkv;
   k.d = P.d;
   k.scale = P.scale;
+  k.hmask = P.hmask;
   for (int h = 0; h < P.V; ++h) k.L[h] = P.L[h];
   k.Q = Q;
   k.K = K;
@@ -365,8 +367,12 @@ spava_status_t run_compress(const Plan& P, const void* Q, const void* K, const v
   cp.scale = P.scale;
   cp.merge_count = merge_count;
   cp.n_merge = merge_count ? P.n_merge : 0;
-  for (int h = 0; h < P.V - 1; ++h) cp.lmax = std::max(cp.lmax, P.L[h]);
-  const dim3 grid(kCompressCtas, P.V - 1, P.Hkv);
+  if (P.ncblk == 0) return SPAVA_OK;   // a host mask that selects no compressed block
+  for (int i = 0; i < P.ncblk; ++i) {
+    cp.blk[i] = P.cblk[i];
+    cp.lmax = std::max(cp.lmax, P.L[P.cblk[i]]);
+  }
+  const dim3 grid(kCompressCtas, P.ncblk, P.Hkv);
   const int smem = compress_smem_bytes(cp.lmax);   // sized to the longest block: two CTAs per SM fit
   const auto* q = static_cast<const __nv_bfloat16*>(Q);
   const auto* k = static_cast<const __nv_bfloat16*>(K);
@@ -588,6 +594,7 @@ spava_status_t spava_score(const spava_problem_t* prob, const void* Q, const voi
   spava_status_t s = make_plan(prob, &P);
   if (s != SPAVA_OK) return s;
   if (P.score_kind != kScoreLinear) return SPAVA_ERR_UNSUPPORTED;   // spava_score_variant
+  if (P.partial) return SPAVA_ERR_UNSUPPORTED;
   return run_score(P, Q, K, qsum, scores, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -596,6 +603,7 @@ spava_status_t spava_score_variant(const spava_problem_t* prob, const void* Q, c
   Plan P;
   spava_status_t s = make_plan(prob, &P);
   if (s != SPAVA_OK) return s;
+  if (P.partial) return SPAVA_ERR_UNSUPPORTED;
   if (P.score_kind == kScoreLinear) {   // the pages' selector needs no workspace
     if (!workspace || ws_bytes < P.ws_total) return SPAVA_ERR_WORKSPACE;
     float* qsum = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + P.ws_qsum);
@@ -612,6 +620,7 @@ spava_status_t spava_select_topk(const spava_problem_t* prob, const float* score
   Plan P;
   spava_status_t s = make_plan(prob, &P);
   if (s != SPAVA_OK) return s;
+  if (P.partial) return SPAVA_ERR_UNSUPPORTED;
   return run_topk(P, scores, idx, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -620,6 +629,7 @@ spava_status_t spava_gather_passing(const spava_problem_t* prob, const void* K, 
   Plan P;
   spava_status_t s = make_plan(prob, &P);
   if (s != SPAVA_OK) return s;
+  if (P.partial) return SPAVA_ERR_UNSUPPORTED;
   return run_gather(P, K, V, idx, Kp, Vp, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -656,6 +666,7 @@ spava_status_t spava_layer_fwd(const spava_problem_t* prob, const void* Q, const
   Plan P;
   spava_status_t s = make_plan(prob, &P);
   if (s != SPAVA_OK) return s;
+  if (P.partial) return SPAVA_ERR_UNSUPPORTED;   // needs the other hosts' passing rows
   if (!Q || !K || !V || !O || !lse) return SPAVA_ERR_INVALID_ARG;
   if (!workspace || ws_bytes < P.ws_total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return SPAVA_ERR_WORKSPACE;
@@ -732,6 +743,7 @@ extern "C" spava_status_t spava_layer_fwd_noalloc(const spava_problem_t* prob, c
   Plan P;
   spava_status_t s = make_plan(prob, &P);
   if (s != SPAVA_OK) return s;
+  if (P.partial) return SPAVA_ERR_UNSUPPORTED;
   if (P.ws_total > kStaticScratchBytes) return SPAVA_ERR_WORKSPACE;   // problem too large for it
   if (!Q || !K || !V || !O || !lse) return SPAVA_ERR_INVALID_ARG;
   void* base = nullptr;

@@ -32,7 +32,8 @@ class _Problem(ctypes.Structure):
                 ("block_lens", ctypes.POINTER(ctypes.c_int32)), ("query_len", ctypes.c_int32),
                 ("lp", ctypes.c_int32), ("num_q_heads", ctypes.c_int32),
                 ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
-                ("softmax_scale", ctypes.c_float), ("score_kind", ctypes.c_int32)]
+                ("softmax_scale", ctypes.c_float), ("score_kind", ctypes.c_int32),
+                ("host_mask", ctypes.c_uint32)]
 
 
 class _Sizes(ctypes.Structure):
@@ -88,26 +89,36 @@ def _check(fn: str, code: int) -> None:
 class Problem:
     """One layer's problem: H physical hosts (2H context blocks), anchor
     length la, context block lengths, query length lq, passing length lp,
-    query/KV heads and head_dim."""
+    query/KV heads and head_dim.  host_mask (0 = all) selects the virtual
+    hosts a call computes (bit h: host h; the anchor rows go with bit 0)."""
 
     def __init__(self, num_hosts: int, anchor_len: int, block_lens: Sequence[int],
                  query_len: int, lp: int, num_q_heads: int, num_kv_heads: int,
-                 head_dim: int, softmax_scale: float = 0.0, score_kind: str = "linear"):
+                 head_dim: int, softmax_scale: float = 0.0, score_kind: str = "linear",
+                 host_mask: int = 0):
         self.num_hosts, self.anchor_len = int(num_hosts), int(anchor_len)
         self.block_lens = [int(x) for x in block_lens]
         self.query_len, self.lp = int(query_len), int(lp)
         self.num_q_heads, self.num_kv_heads = int(num_q_heads), int(num_kv_heads)
         self.head_dim, self.softmax_scale = int(head_dim), float(softmax_scale)
         self.score_kind = score_kind
+        self.host_mask = int(host_mask)
         self._arr = (ctypes.c_int32 * max(1, len(self.block_lens)))(*self.block_lens)
         self._c = _Problem(self.num_hosts, self.anchor_len, self._arr, self.query_len, self.lp,
                            self.num_q_heads, self.num_kv_heads, self.head_dim, self.softmax_scale,
-                           SCORE_KINDS[score_kind])
+                           SCORE_KINDS[score_kind], self.host_mask)
 
     @classmethod
-    def from_workload(cls, wl, score_kind: str = "linear") -> "Problem":
+    def from_workload(cls, wl, score_kind: str = "linear", host_mask: int = 0) -> "Problem":
         return cls(wl.num_hosts, wl.anchor_len, wl.block_lens, wl.query_len, wl.lp,
-                   wl.num_q_heads, wl.num_kv_heads, wl.head_dim, score_kind=score_kind)
+                   wl.num_q_heads, wl.num_kv_heads, wl.head_dim, score_kind=score_kind,
+                   host_mask=host_mask)
+
+    def with_hosts(self, host_mask: int) -> "Problem":
+        """The same problem restricted to the virtual hosts of host_mask."""
+        return Problem(self.num_hosts, self.anchor_len, self.block_lens, self.query_len, self.lp,
+                       self.num_q_heads, self.num_kv_heads, self.head_dim, self.softmax_scale,
+                       self.score_kind, host_mask)
 
     @property
     def ref(self):
