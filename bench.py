@@ -267,13 +267,13 @@ def run_reference(args, wl):
     return 0
 
 
-def config_of(wl, n):
+def config_of(wl, n, parallelism="replicas (one independent layer per GPU)"):
     return {"workload": wl.name, "seq_len": n, "num_hosts": wl.num_hosts,
             "virtual_hosts": 2 * wl.num_hosts, "anchor_len": wl.anchor_len,
             "block_lens": sorted(set(wl.block_lens)) if len(set(wl.block_lens)) == 1 else wl.block_lens,
             "query_len": wl.query_len, "lp": wl.lp, "q_heads": wl.num_q_heads,
             "kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
-            "parallelism": "replicas (one independent layer per GPU)",
+            "parallelism": parallelism,
             "l2": "3 rotating input sets, each larger than L2"}
 
 
@@ -319,11 +319,26 @@ def run_gpu(args, wl):
     ws = torch.empty(sz["workspace_bytes"], dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def layer(k):
-        x = sets[k % 3]
-        spava.layer_fwd(p, x["Q"], x["K"], x["V"], O, lse, ws, stream=stream)
+    if args.mode == "hosts":
+        # the pages' split: rank r computes the virtual hosts of its mask and
+        # the ranks exchange passing rows and query partials (hosts.py)
+        from sparse_approximate_attention_b200 import hosts
+        sharded = hosts.HostShardedLayer(p, world, rank, dev)
+        q = sharded.q
 
-    launches_per_step = 2   # compression (or the zeroing of the merge counters when lp = 0) + attention
+        def layer(k):
+            x = sets[k % 3]
+            sharded.forward(x["Q"], x["K"], x["V"], O, lse, stream=stream)
+
+        launches_per_step = 3 if lp > 0 else 2   # compression, attention, merge (collectives are NCCL's)
+    else:
+        q = p
+
+        def layer(k):
+            x = sets[k % 3]
+            spava.layer_fwd(p, x["Q"], x["K"], x["V"], O, lse, ws, stream=stream)
+
+        launches_per_step = 2   # compression (or the zeroing of the merge counters when lp = 0) + attention
 
     for i in range(args.warmup):
         layer(i)
@@ -346,7 +361,8 @@ def run_gpu(args, wl):
     err = spava.device_error()
     assert err == 0, f"device error word {err}"
     ms_per_step = elapsed_ms / args.steps
-    value = world * n / (ms_per_step / 1000.0)
+    # replicas: every rank processes a layer; hosts: the ranks process one together
+    value = (1 if args.mode == "hosts" else world) * n / (ms_per_step / 1000.0)
 
     # ---------------- the kernels on their own (same launch configuration as in the layer)
     qsum = torch.empty(hkv, d, dtype=f32, device=dev)
@@ -358,12 +374,12 @@ def run_gpu(args, wl):
     lse_part = torch.empty(V, hq, lq, dtype=f32, device=dev)
     stage_ms = {}
     if lp > 0:
-        comp = lambda k: spava.compress(p, sets[k % 3]["Q"], sets[k % 3]["K"], sets[k % 3]["V"], qsum, scores,
+        comp = lambda k: spava.compress(q, sets[k % 3]["Q"], sets[k % 3]["K"], sets[k % 3]["V"], qsum, scores,
                                         idx, Kp, Vp, stream=stream)
         for k in range(3):
             comp(k)
         stage_ms["compress"] = timed_loop(comp, args.steps, stream, dev)
-    attn = lambda k: spava.attn_fwd(p, sets[k % 3]["Q"], sets[k % 3]["K"], sets[k % 3]["V"],
+    attn = lambda k: spava.attn_fwd(q, sets[k % 3]["Q"], sets[k % 3]["K"], sets[k % 3]["V"],
                                     Kp if lp else None, Vp if lp else None, O, lse, O_part, lse_part,
                                     stream=stream)
     for k in range(3):
@@ -376,7 +392,7 @@ def run_gpu(args, wl):
     stage_ms["merge"] = timed_loop(merge, args.steps, stream, dev)
     assert spava.device_error() == 0
 
-    if args.no_e2e:
+    if args.no_e2e or args.mode == "hosts":
         e2e_ms, e2e_value, h2d, d2h = None, None, 0, 0
     else:
         e2e_ms, e2e_value, h2d, d2h = e2e_measure(p, host_inp, sets, O, lse, ws, stream, dev,
@@ -384,7 +400,7 @@ def run_gpu(args, wl):
     if rank != 0:
         return 0
     return report(args, wl, sz, world, n, ms_per_step, elapsed_ms, value, stage_ms, attn_region_s, e2e_ms,
-                  e2e_value, h2d, d2h, launches_per_step, clk, clk_attn, host_inp)
+                  e2e_value, h2d, d2h, launches_per_step, clk, clk_attn, host_inp, q.sizes())
 
 
 def e2e_measure(p, host_inp, sets, O, lse, ws, stream, dev, world, n, steps):
@@ -445,7 +461,7 @@ def e2e_measure(p, host_inp, sets, O, lse, ws, stream, dev, world, n, steps):
 
 
 def report(args, wl, sz, world, n, ms_per_step, elapsed_ms, value, stage_ms, attn_region_s, e2e_ms,
-           e2e_value, h2d, d2h, launches_per_step, clk, clk_attn, host_inp):
+           e2e_value, h2d, d2h, launches_per_step, clk, clk_attn, host_inp, rank_sz=None):
     hq, hkv, d, V, lq, lp = (wl.num_q_heads, wl.num_kv_heads, wl.head_dim, 2 * wl.num_hosts,
                              wl.query_len, wl.lp)
     pk, src = peaks()
@@ -456,7 +472,9 @@ def report(args, wl, sz, world, n, ms_per_step, elapsed_ms, value, stage_ms, att
     # at the burst clock, a longer one settles under the power cap
     sustained_region = attn_region_s >= 1.0
     peak_tf = sustained if sustained_region else burst
-    flops = sz["attn_flops"]
+    hosts_mode = args.mode == "hosts"
+    # the attention launch of this rank: all rows, or the rows of its host mask
+    flops = (rank_sz or sz)["attn_flops"]
     attn_tf = flops / (stage_ms["attn"] / 1000.0) / 1e12
     S, P = sz["score_cols"], sz["passing_rows"]
     by = {
@@ -483,11 +501,15 @@ def report(args, wl, sz, world, n, ms_per_step, elapsed_ms, value, stage_ms, att
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "strong" if hosts_mode else "weak", "vs_baseline": None,
+        "dtype": "bf16",
         "data": "synthetic (seeded long-video-shaped Q/K/V: rank-16 per-frame K/V + noise, "
                 "query block correlated with 2% of context keys)",
-        "config": config_of(wl, n),
-        "tflops_layer": round(flops / (ms_per_step / 1000.0) / 1e12, 1),
+        "config": config_of(wl, n, (f"hosts over {world} GPU(s): rank r holds virtual hosts p and 2H-1-p "
+                                    f"for its physical hosts p (p % {world} == r); NCCL all-gather of passing "
+                                    f"rows and query partials") if hosts_mode else
+                            "replicas (one independent layer per GPU)"),
+        "tflops_layer": round(sz["attn_flops"] / (ms_per_step / 1000.0) / 1e12, 1),
         "roofline": {"bound": "tensor", "kernel": f"attn_kernel<{d}>", "achieved": round(attn_tf, 1),
                      "peak": peak_tf, "unit": "TFLOP/s", "frac": round(attn_tf / peak_tf, 4),
                      "traffic": committed_traffic(wl.name),
@@ -497,8 +519,10 @@ def report(args, wl, sz, world, n, ms_per_step, elapsed_ms, value, stage_ms, att
                      "frac_of_burst": round(attn_tf / burst, 4), "frac_of_sustained": round(attn_tf / sustained, 4),
                      "algorithmic_flops_per_launch": flops, "clocks": clk_attn.summary()},
         "stages": stage_info,
-        "layer": "spava_layer_fwd: compression launch, then attention with the query-partial merge "
-                 "(programmatic dependent launch)",
+        "layer": ("per rank: spava_compress and spava_attn_fwd with the rank's host mask, all-gathers of "
+                  "passing rows and query partials, spava_lse_merge") if hosts_mode else
+                 ("spava_layer_fwd: compression launch, then attention with the query-partial merge "
+                  "(programmatic dependent launch)"),
         "e2e": None if e2e_ms is None else {
             "value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3),
@@ -525,6 +549,9 @@ def main():
     ap.add_argument("--impl", default="spava", choices=["spava", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--mode", default="replicas", choices=["replicas", "hosts"],
+                    help="replicas: one independent layer per GPU (default); hosts: the pages' split of "
+                         "one layer's virtual hosts over the GPUs")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
