@@ -250,13 +250,6 @@ spava_status_t spava_layer_fwd_noalloc(const spava_problem_t* prob, const void* 
  * kernel gave up; bit 1: the gather met an index outside its block. */
 spava_status_t spava_device_error(uint32_t* code);
 
-/* Test hook, not part of the layer: y[i] = the 2^x approximation that the
- * attention softmax evaluates on the FMA pipe for a share of its
- * exponentials (a Cody-Waite split x = i + f, a cubic least-squares fit of
- * 2^f on [-1/2, 1/2], 2^i added to the exponent; exactly 0 below -126).
- * x, y: device float arrays of n elements, n even, 16-byte aligned. */
-spava_status_t spava_debug_exp2_poly(const float* x, float* y, int64_t n, spava_stream_t stream);
-
 /* Human-readable name of a status code (static string). */
 const char* spava_status_string(spava_status_t status);
 

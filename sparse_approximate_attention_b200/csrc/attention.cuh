@@ -26,8 +26,8 @@
 //              softmax runs
 //   warps 2-3  idle (they complete warpgroup 0)
 //   warps 4-7  softmax of Q0, warps 8-11 softmax of Q1: one thread per row,
-//              online softmax in the exp2 domain (3/8 of the exponentials on
-//              the FMA pipe, packed f32x2 arithmetic), lazy rescale of O (only
+//              online softmax in the exp2 domain (exponentials on MUFU,
+//              packed f32x2 arithmetic elsewhere), lazy rescale of O (only
 //              when the row max grows by more than 2^8), P written back to
 //              TMEM as bf16 over S
 // TMEM columns: O0 [0, D), O1 [128, 128 + D), S0/P0 [256, 384), S1/P1 [384, 512).
@@ -459,12 +459,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1)
         for (int u = 0; u < 32; ++u) {
           const int i = 32 * half + u;
           const float2 y = __ffma2_rn(x[i], sl22, neg2);
-          float2 pe;
-          if ((i & 7) < 3) {   // three pairs in eight on the FMA pipe, the rest on MUFU
-            pe = exp2_poly2(y);
-          } else {
-            pe = make_float2(ex2_approx(y.x), ex2_approx(y.y));
-          }
+          const float2 pe = make_float2(ex2_approx(y.x), ex2_approx(y.y));
           acc[i & 3] = __fadd2_rn(acc[i & 3], pe);
           pk[u] = pack_bf16x2(pe.x, pe.y);
         }

@@ -281,27 +281,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// 2^x for a pair of values on the FMA pipe (packed f32x2 arithmetic), used
-// for a share of the softmax exponentials so that the MUFU unit is not the
-// only source.  x = i + f with i = round(x) (via the 1.5*2^23 rounding
-// constant) and f in [-0.5, 0.5]; 2^f by a cubic fitted by least squares to
-// 2^f in fp64 at 2000 Chebyshev nodes of [-0.5, 0.5] (max relative error
-// 1.1e-4 evaluated in fp32, below bf16's 2^-9); 2^i by adding i to the
-// exponent field.  Valid for x <= 64; exactly 0 for x < -126 (and -inf).
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  const float2 kRound = make_float2(12582912.0f, 12582912.0f);
-  const float2 kUnround = make_float2(-12582912.0f, -12582912.0f);
-  const float2 r = __fadd2_rn(x, kRound);
-  const float2 f = __ffma2_rn(__fadd2_rn(r, kUnround), make_float2(-1.0f, -1.0f), x);
-  float2 p = __ffma2_rn(f, make_float2(0.05592203512787819f, 0.05592203512787819f),
-                        make_float2(0.24264007806777954f, 0.24264007806777954f));
-  p = __ffma2_rn(p, f, make_float2(0.6931210160255432f, 0.6931210160255432f));
-  p = __ffma2_rn(p, f, make_float2(0.9999244809150696f, 0.9999244809150696f));
-  const float y0 = __int_as_float(__float_as_int(p.x) + (__float_as_int(r.x) << 23));
-  const float y1 = __int_as_float(__float_as_int(p.y) + (__float_as_int(r.y) << 23));
-  return make_float2(x.x < -126.0f ? 0.0f : y0, x.y < -126.0f ? 0.0f : y1);
-}
-
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));

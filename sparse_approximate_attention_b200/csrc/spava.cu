@@ -548,17 +548,6 @@ spava_status_t run_layer(const Plan& P, uint8_t* ws, const void* Q, const void* 
 
 }  // namespace
 
-namespace {
-
-// y[i] = the attention softmax's FMA-pipe 2^x (exp2_poly2) applied to x[i];
-// n even.  Test hook for the approximation's error bound.
-__global__ void exp2_poly_kernel(const float2* __restrict__ x, float2* __restrict__ y, int64_t npairs) {
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < npairs;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
-    y[i] = exp2_poly2(x[i]);
-}
-
-}  // namespace
 
 // ===================================================================== C ABI
 extern "C" {
@@ -681,16 +670,6 @@ spava_status_t spava_device_error(uint32_t* code) {
   if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess) return SPAVA_ERR_CUDA;
   *code = v;
   return SPAVA_OK;
-}
-
-spava_status_t spava_debug_exp2_poly(const float* x, float* y, int64_t n, spava_stream_t stream) {
-  if (!x || !y || n < 0 || (n & 1) || !aligned16(x) || !aligned16(y)) return SPAVA_ERR_INVALID_ARG;
-  if (n == 0) return SPAVA_OK;
-  const int64_t npairs = n / 2;
-  const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((npairs + 255) / 256, 148 * 8));
-  exp2_poly_kernel<<<static_cast<unsigned>(blocks), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-      reinterpret_cast<const float2*>(x), reinterpret_cast<float2*>(y), npairs);
-  return last_launch();
 }
 
 const char* spava_status_string(spava_status_t status) {

@@ -59,7 +59,6 @@ _SIGS = {
     "spava_layer_fwd": [_PP, _VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_size_t, _VP],
     "spava_device_error": [ctypes.POINTER(ctypes.c_uint32)],
     "spava_layer_fwd_noalloc": [_PP, _VP, _VP, _VP, _VP, _VP, _VP],
-    "spava_debug_exp2_poly": [_VP, _VP, ctypes.c_int64, _VP],
 }
 
 
@@ -306,14 +305,3 @@ def layer_fwd_noalloc(p: Problem, Q, K, V, O, lse, stream=None):
     _check("spava_layer_fwd_noalloc", lib().spava_layer_fwd_noalloc(
         p.ref, _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(lse), _stream(stream)))
     return O, lse
-
-
-def debug_exp2_poly(x, y=None, stream=None):
-    """The attention softmax's FMA-pipe 2^x approximation applied to x
-    (float32, even length, on the GPU) -- a test hook for its error bound."""
-    if x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous() or x.numel() % 2:
-        raise ValueError("x: expected a contiguous cuda float32 tensor of even length")
-    y = torch.empty_like(x) if y is None else y
-    _need(y, torch.float32, tuple(x.shape), "y")
-    _check("spava_debug_exp2_poly", lib().spava_debug_exp2_poly(_ptr(x), _ptr(y), x.numel(), _stream(stream)))
-    return y
