@@ -250,6 +250,15 @@ spava_status_t spava_layer_fwd_noalloc(const spava_problem_t* prob, const void* 
  * kernel gave up; bit 1: the gather met an index outside its block. */
 spava_status_t spava_device_error(uint32_t* code);
 
+/* Test hook, not part of the layer: one thread of a one-CTA kernel waits on
+ * an mbarrier that nothing completes, through the same bounded waits the
+ * kernels use, with a limit of limit_ns (0 < limit_ns <= 4 s).  The wait gives
+ * up, raises the CTA's abort flag and sets bit 0 of the device error word;
+ * then the drain wait gives up too.  out (device, 4 x int64): the wait's
+ * result (0), the abort flag (1), the drain's result (0), the nanoseconds
+ * both took.  The context stays usable. */
+spava_status_t spava_debug_wait_timeout(int64_t* out, uint64_t limit_ns, spava_stream_t stream);
+
 /* Human-readable name of a status code (static string). */
 const char* spava_status_string(spava_status_t status);
 

@@ -549,6 +549,31 @@ spava_status_t run_layer(const Plan& P, uint8_t* ws, const void* Q, const void* 
 }  // namespace
 
 
+namespace {
+
+// Test hook: one thread waits on an mbarrier that nothing will complete, with
+// the kernels' own bounded waits and a short limit.  out[0] = what mbar_wait
+// returned, out[1] = the abort flag it left, out[2] = what mbar_wait_drain
+// returned, out[3] = nanoseconds the two waits took.
+__global__ void wait_timeout_kernel(int64_t* out, uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x != 0) return;
+  const uint32_t b = smem_u32(&bar);
+  mbar_init(b, 1);
+  abort_flag = 0;
+  fence_barrier_init();
+  const uint64_t t0 = globaltimer_ns();
+  const bool w = mbar_wait(b, 0, &abort_flag, limit_ns);
+  const bool d = mbar_wait_drain(b, 0, limit_ns);
+  out[0] = w;
+  out[1] = abort_flag;
+  out[2] = d;
+  out[3] = static_cast<int64_t>(globaltimer_ns() - t0);
+}
+
+}  // namespace
+
 // ===================================================================== C ABI
 extern "C" {
 
@@ -670,6 +695,12 @@ spava_status_t spava_device_error(uint32_t* code) {
   if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess) return SPAVA_ERR_CUDA;
   *code = v;
   return SPAVA_OK;
+}
+
+spava_status_t spava_debug_wait_timeout(int64_t* out, uint64_t limit_ns, spava_stream_t stream) {
+  if (!out || limit_ns == 0 || limit_ns > kWaitLimitNs) return SPAVA_ERR_INVALID_ARG;
+  wait_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(out, limit_ns);
+  return last_launch();
 }
 
 const char* spava_status_string(spava_status_t status) {

@@ -59,6 +59,7 @@ _SIGS = {
     "spava_layer_fwd": [_PP, _VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_size_t, _VP],
     "spava_device_error": [ctypes.POINTER(ctypes.c_uint32)],
     "spava_layer_fwd_noalloc": [_PP, _VP, _VP, _VP, _VP, _VP, _VP],
+    "spava_debug_wait_timeout": [_VP, ctypes.c_uint64, _VP],
 }
 
 
@@ -305,3 +306,11 @@ def layer_fwd_noalloc(p: Problem, Q, K, V, O, lse, stream=None):
     _check("spava_layer_fwd_noalloc", lib().spava_layer_fwd_noalloc(
         p.ref, _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(lse), _stream(stream)))
     return O, lse
+
+
+def debug_wait_timeout(limit_ns: int, stream=None):
+    """Test hook: a bounded mbarrier wait that runs out after limit_ns.
+    Returns (wait result, abort flag, drain result, elapsed ns)."""
+    out = torch.zeros(4, dtype=torch.int64, device="cuda")
+    _check("spava_debug_wait_timeout", lib().spava_debug_wait_timeout(_ptr(out), int(limit_ns), _stream(stream)))
+    return tuple(int(v) for v in out.cpu().tolist())

@@ -369,3 +369,23 @@ def test_layer_with_score_variant(kind):
     heads = list(range(wl.num_q_heads))
     got_rows, o_ref, l_ref = oracle.rows_fwd(lay, inp["Q"], inp["K"], inp["V"], ref_idx, rows, heads)
     check_rows(lay, inp, sel, affected, got_rows, heads, to_np(O).astype(np.float64), to_np(lse), o_ref, l_ref)
+
+
+def test_bounded_wait_gives_up_reports_and_leaves_the_context_usable():
+    """A wait on an mbarrier that nothing completes (the kernels' own bounded
+    waits, with a 2 ms limit) gives up, raises the abort flag and sets the
+    device error word; the next device_error() reads it and clears it, and the
+    layer then still runs correctly."""
+    assert spava.device_error() == 0
+    w, ab, dr, ns = spava.debug_wait_timeout(2_000_000)
+    assert (w, ab, dr) == (0, 1, 0)
+    assert 3_000_000 <= ns < 1_000_000_000
+    assert spava.device_error() == 1
+    assert spava.device_error() == 0
+    wl, lay, inp, ref = _case("tiny")
+    d = _dev(inp)
+    O, lse = spava.layer_fwd(spava.Problem.from_workload(wl), d["Q"], d["K"], d["V"])
+    torch.cuda.synchronize()
+    _no_device_error()
+    assert max_err(to_np(O).astype(np.float64), ref["O"]) <= O_TOL
+    assert max_err(to_np(lse), ref["lse"]) <= LSE_TOL
