@@ -6,13 +6,14 @@
 // review), "What carries the argument": each context block is compressed to
 // its top-lp key-value pairs ranked by Q_qr K^T and gathered by later hosts.
 //
-// One thread-block cluster of kCompressCtas CTAs per (block h < V-1, KV head)
-// (all such blocks, or those a host mask selects),
+// One thread-block cluster of nc CTAs (4 or 8, chosen at launch so that the
+// grid fits the GPU in one wave when it can) per (block h < V-1, KV head) (all such
+// blocks, or those a host mask selects),
 // for blocks of up to kCompressMaxBlock keys:
 //   1. each CTA sums a slice of the query block's (row, head) pairs of the KV
 //      group; the slices are added in rank order through distributed shared
 //      memory, so every CTA holds the same qsum = scale * sum q;
-//   2. each CTA streams its 1/kCompressCtas slice of K^(h) once (16-byte
+//   2. each CTA streams its 1/nc slice of K^(h) once (16-byte
 //      loads, the first ones issued before step 1) and turns the scores into
 //      order-preserving 32-bit keys (the scores are also written out); it
 //      then copies its slice's keys into every CTA of the cluster, so that
@@ -35,16 +36,24 @@
 
 namespace spava {
 
-constexpr int kCompressCtas = 8;
+constexpr int kCompressMinCtas = 4;    // cluster sizes: 4 or 8 (16, a non-portable size, was
+constexpr int kCompressMaxCtas = 8;    // measured slower on small problems: 31 us against 27)
 constexpr int kCompressThreads = 512;
 constexpr int kCompressWarps = kCompressThreads / 32;
-constexpr int kCompressMaxBlock = 24576;                               // keys per block
-constexpr int kCompressMaxSlice = kCompressMaxBlock / kCompressCtas;   // keys per CTA
+constexpr int kCompressMaxBlock = 24576;   // keys per block
+static_assert(kCompressMaxBlock <= 65536, "kept keys pack their block index and rank in 16 bits each");
 
-// Dynamic shared memory of a launch whose longest compressed block has
-// lmax keys: every key of the block, then this CTA's kept keys and their ranks.
-__host__ __device__ constexpr int compress_smem_bytes(int lmax) {
-  return 4 * ((lmax + 3) / 4 * 4) + 8 * ((lmax + kCompressCtas - 1) / kCompressCtas);
+// Scratch shared by two phases: the query sum's per-warp partials (step 1,
+// kCompressWarps x 128 floats at most) and the radix select's per-warp
+// histograms (step 3, kCompressWarps x 256 counts).
+constexpr int kCompressScratchBytes = kCompressWarps * 256 * 4;
+
+// Dynamic shared memory of a launch with clusters of nc CTAs whose longest
+// compressed block has lmax keys: every key of the block, this CTA's kept
+// keys (block index and rank packed in 32 bits; at most one slice), then the
+// scratch.
+__host__ __device__ constexpr int compress_smem_bytes(int lmax, int nc) {
+  return 4 * ((lmax + 3) / 4 * 4) + 4 * (((lmax + nc - 1) / nc + 3) / 4 * 4) + kCompressScratchBytes;
 }
 
 struct CompressParams {
@@ -64,7 +73,7 @@ struct CompressParams {
 };
 
 template <int D>
-__global__ void __cluster_dims__(kCompressCtas, 1, 1) __launch_bounds__(kCompressThreads, 2)
+__global__ void __launch_bounds__(kCompressThreads, 2)
     compress_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
                     const __nv_bfloat16* __restrict__ V, float* __restrict__ qsum_out,
                     float* __restrict__ scores, int32_t* __restrict__ idx,
@@ -74,12 +83,13 @@ __global__ void __cluster_dims__(kCompressCtas, 1, 1) __launch_bounds__(kCompres
   constexpr int kRowsPerIter = kCompressThreads / kParts;
   extern __shared__ uint8_t dsm[];
   uint32_t* keys = reinterpret_cast<uint32_t*>(dsm);                                  // [L] whole block
-  int32_t* sel_j = reinterpret_cast<int32_t*>(dsm + 4 * ((p.lmax + 3) / 4 * 4));     // [slice]
-  int32_t* sel_pos = sel_j + (p.lmax + kCompressCtas - 1) / kCompressCtas;           // [slice]
-  __shared__ float part_q[kCompressWarps][D];
+  uint32_t* sel = reinterpret_cast<uint32_t*>(dsm + 4 * ((p.lmax + 3) / 4 * 4));    // [slice]: (rank << 16) | j
+  const int nc = static_cast<int>(gridDim.x);   // the cluster: one per (block, KV head)
+  uint8_t* scratch = reinterpret_cast<uint8_t*>(sel + ((p.lmax + nc - 1) / nc + 3) / 4 * 4);
+  float (*part_q)[D] = reinterpret_cast<float (*)[D]>(scratch);              // step 1
+  uint32_t (*hist)[256] = reinterpret_cast<uint32_t (*)[256]>(scratch);     // step 3, one per warp
   __shared__ float slice_q[D];
   __shared__ float qs_full[D];
-  __shared__ uint32_t hist[kCompressWarps][256];   // one histogram per warp
   __shared__ uint32_t tot[256];
   __shared__ uint64_t warp_tot[32];
   __shared__ uint32_t s_prefix, s_k;
@@ -96,8 +106,8 @@ __global__ void __cluster_dims__(kCompressCtas, 1, 1) __launch_bounds__(kCompres
   if (p.merge_count != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && kv == 0)
     for (int i = tid; i < p.n_merge; i += kCompressThreads) p.merge_count[i] = 0;
   const int L = p.L[h], kk = p.k[h];
-  const int j0 = static_cast<int>((static_cast<int64_t>(L) * rank) / kCompressCtas);
-  const int j1 = static_cast<int>((static_cast<int64_t>(L) * (rank + 1)) / kCompressCtas);
+  const int j0 = static_cast<int>((static_cast<int64_t>(L) * rank) / nc);
+  const int j1 = static_cast<int>((static_cast<int64_t>(L) * (rank + 1)) / nc);
   const int n = j1 - j0;   // keys of this CTA's slice
   const int pc = tid % kParts, lr = tid / kParts;
 
@@ -120,8 +130,8 @@ __global__ void __cluster_dims__(kCompressCtas, 1, 1) __launch_bounds__(kCompres
   // ---- 1. qsum for this KV group
   {
     const int total = p.lq * p.G;
-    const int r0 = static_cast<int>((static_cast<int64_t>(total) * rank) / kCompressCtas);
-    const int r1 = static_cast<int>((static_cast<int64_t>(total) * (rank + 1)) / kCompressCtas);
+    const int r0 = static_cast<int>((static_cast<int64_t>(total) * rank) / nc);
+    const int r1 = static_cast<int>((static_cast<int64_t>(total) * (rank + 1)) / nc);
     float acc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.f;
@@ -160,7 +170,7 @@ __global__ void __cluster_dims__(kCompressCtas, 1, 1) __launch_bounds__(kCompres
     cluster.sync();
     for (int c = tid; c < D; c += kCompressThreads) {
       float s = 0.f;
-      for (int r = 0; r < kCompressCtas; ++r) s += cluster.map_shared_rank(slice_q, r)[c];
+      for (int r = 0; r < nc; ++r) s += cluster.map_shared_rank(slice_q, r)[c];
       qs_full[c] = s * p.scale;
       if (h == 0 && rank == 0) qsum_out[kv * D + c] = s * p.scale;
     }
@@ -194,8 +204,8 @@ __global__ void __cluster_dims__(kCompressCtas, 1, 1) __launch_bounds__(kCompres
     }
   }
   __syncthreads();
-  for (int r = 1; r < kCompressCtas; ++r) {   // this slice's keys into every other CTA
-    uint32_t* dst = cluster.map_shared_rank(keys, (rank + r) % kCompressCtas);
+  for (int r = 1; r < nc; ++r) {   // this slice's keys into every other CTA
+    uint32_t* dst = cluster.map_shared_rank(keys, (rank + r) % nc);
     for (int i = tid; i < n; i += kCompressThreads) dst[j0 + i] = keys[j0 + i];
   }
   cluster.sync();   // every CTA holds the block's keys; the last access to peer shared memory
@@ -303,8 +313,7 @@ __global__ void __cluster_dims__(kCompressCtas, 1, 1) __launch_bounds__(kCompres
       }
       if (pos >= 0) {
         out[pos] = j0 + i;
-        sel_j[lsel] = j0 + i;
-        sel_pos[lsel] = pos;
+        sel[lsel] = (static_cast<uint32_t>(pos) << 16) | static_cast<uint32_t>(j0 + i);
         ++lsel;
       }
     }
@@ -324,7 +333,7 @@ __global__ void __cluster_dims__(kCompressCtas, 1, 1) __launch_bounds__(kCompres
       for (int u = 0; u < 4; ++u) {
         const int s = sb + u * kRowsPerIter;
         if (s < nsel) {
-          const int64_t src = static_cast<int64_t>(p.start[h]) + sel_j[s];
+          const int64_t src = static_cast<int64_t>(p.start[h]) + (sel[s] & 0xFFFFu);
           kx[u] = *reinterpret_cast<const uint4*>(K + (src * p.Hkv + kv) * D + pc * 8);
           vx[u] = *reinterpret_cast<const uint4*>(V + (src * p.Hkv + kv) * D + pc * 8);
         }
@@ -333,7 +342,7 @@ __global__ void __cluster_dims__(kCompressCtas, 1, 1) __launch_bounds__(kCompres
       for (int u = 0; u < 4; ++u) {
         const int s = sb + u * kRowsPerIter;
         if (s < nsel) {
-          const int64_t dst = off + sel_pos[s];
+          const int64_t dst = off + (sel[s] >> 16);
           *reinterpret_cast<uint4*>(Kp + (dst * p.Hkv + kv) * D + pc * 8) = kx[u];
           *reinterpret_cast<uint4*>(Vp + (dst * p.Hkv + kv) * D + pc * 8) = vx[u];
         }

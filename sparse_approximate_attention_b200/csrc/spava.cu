@@ -70,6 +70,8 @@ struct DeviceSetup {
   bool done = false;
   spava_status_t status = SPAVA_OK;
   int sm_count = 148;
+  int smem_per_sm = 228 * 1024;      // shared memory of one SM
+  int compress_static[2] = {0, 0};   // static shared memory of compress_kernel<64>, <128>
 };
 std::mutex g_setup_mu;
 DeviceSetup g_setup[kMaxDevices];
@@ -100,6 +102,8 @@ spava_status_t device_setup(const DeviceSetup** out) {
   if (!s.done) {
     int n = 0;
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0) s.sm_count = n;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) == cudaSuccess && n > 0)
+      s.smem_per_sm = n;
     spava_status_t st = setup_attn<128>();
     if (st == SPAVA_OK) st = setup_attn<64>();
     if (st == SPAVA_OK &&
@@ -108,13 +112,18 @@ spava_status_t device_setup(const DeviceSetup** out) {
          cudaFuncSetAttribute(colsum_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               ColsumCfg<64>::kSmemBytes) != cudaSuccess))
       st = SPAVA_ERR_CUDA;
-    const int csmem = compress_smem_bytes(kCompressMaxBlock);
+    const int csmem = compress_smem_bytes(kCompressMaxBlock, kCompressMinCtas);
     if (st == SPAVA_OK &&
         (cudaFuncSetAttribute(compress_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, csmem) !=
              cudaSuccess ||
          cudaFuncSetAttribute(compress_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, csmem) !=
              cudaSuccess))
       st = SPAVA_ERR_CUDA;
+    cudaFuncAttributes fa;
+    if (st == SPAVA_OK && cudaFuncGetAttributes(&fa, compress_kernel<64>) == cudaSuccess)
+      s.compress_static[0] = static_cast<int>(fa.sharedSizeBytes);
+    if (st == SPAVA_OK && cudaFuncGetAttributes(&fa, compress_kernel<128>) == cudaSuccess)
+      s.compress_static[1] = static_cast<int>(fa.sharedSizeBytes);
     s.status = st;
     s.done = true;
   }
@@ -334,9 +343,14 @@ bool compress_fits(const Plan& P) {
   return true;
 }
 
-// Steps 1-3 in one launch: one cluster of kCompressCtas CTAs per (block, KV
-// head).  merge_count (may be null): the following attention launch's merge
+// Steps 1-3 in one launch: one cluster of nc CTAs per (block, KV head).
+// merge_count (may be null): the following attention launch's merge
 // counters, zeroed by this launch.
+//
+// nc: 8 if the grid of 8-CTA clusters fits the GPU in one wave (two CTAs per
+// SM when the shared memory allows it), else 4, so that as many CTAs as
+// possible stream their slice of K at the same time.  The K stream and the
+// gather shrink with nc, the key broadcast and the local select do not.
 spava_status_t run_compress(const Plan& P, const void* Q, const void* K, const void* V, float* qsum,
                             float* scores, int32_t* idx, void* Kp, void* Vp, int32_t* merge_count,
                             cudaStream_t st) {
@@ -372,17 +386,39 @@ spava_status_t run_compress(const Plan& P, const void* Q, const void* K, const v
     cp.blk[i] = P.cblk[i];
     cp.lmax = std::max(cp.lmax, P.L[P.cblk[i]]);
   }
-  const dim3 grid(kCompressCtas, P.ncblk, P.Hkv);
-  const int smem = compress_smem_bytes(cp.lmax);   // sized to the longest block: two CTAs per SM fit
+  const int pairs = P.ncblk * P.Hkv;
+  int nc = kCompressMinCtas;
+  for (int c = kCompressMaxCtas; c > kCompressMinCtas; c /= 2) {
+    // a CTA's shared memory: dynamic + static + the 1 KB the system reserves per CTA
+    const int cta_bytes = compress_smem_bytes(cp.lmax, c) + ds->compress_static[P.d == 128 ? 1 : 0] + 1024;
+    const int per_sm = std::min(2, std::max(1, ds->smem_per_sm / cta_bytes));
+    if (static_cast<int64_t>(pairs) * c <= static_cast<int64_t>(per_sm) * ds->sm_count) {
+      nc = c;
+      break;
+    }
+  }
+  const int smem = compress_smem_bytes(cp.lmax, nc);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(nc);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(static_cast<unsigned>(nc), static_cast<unsigned>(P.ncblk), static_cast<unsigned>(P.Hkv));
+  cfg.blockDim = dim3(kCompressThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   const auto* q = static_cast<const __nv_bfloat16*>(Q);
   const auto* k = static_cast<const __nv_bfloat16*>(K);
   const auto* v = static_cast<const __nv_bfloat16*>(V);
   auto* kp = static_cast<__nv_bfloat16*>(Kp);
   auto* vp = static_cast<__nv_bfloat16*>(Vp);
-  if (P.d == 128)
-    compress_kernel<128><<<grid, kCompressThreads, smem, st>>>(q, k, v, qsum, scores, idx, kp, vp, cp);
-  else
-    compress_kernel<64><<<grid, kCompressThreads, smem, st>>>(q, k, v, qsum, scores, idx, kp, vp, cp);
+  const cudaError_t e = P.d == 128
+                            ? cudaLaunchKernelEx(&cfg, compress_kernel<128>, q, k, v, qsum, scores, idx, kp, vp, cp)
+                            : cudaLaunchKernelEx(&cfg, compress_kernel<64>, q, k, v, qsum, scores, idx, kp, vp, cp);
+  if (e != cudaSuccess) return SPAVA_ERR_CUDA;
   return last_launch();
 }
 
