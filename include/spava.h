@@ -259,6 +259,19 @@ spava_status_t spava_device_error(uint32_t* code);
  * both took.  The context stays usable. */
 spava_status_t spava_debug_wait_timeout(int64_t* out, uint64_t limit_ns, spava_stream_t stream);
 
+/* Test hook, not part of the layer: spava_attn_fwd with one key tile left
+ * unloaded.  The producer of every CTA skips its key tile skip_k_tile (>= 0),
+ * and every wait of the launch gives up after limit_ns (0 < limit_ns <= 4 s)
+ * instead of 4 s, so the CTAs that reach that tile take the kernel's abort
+ * path: the MMA warp's wait runs out, the abort flag stops the other roles,
+ * the copies and MMAs in flight are drained (bounded), TMEM is freed and bit
+ * 0 of the device error word is set.  The outputs of the call are invalid;
+ * the context stays usable. */
+spava_status_t spava_debug_attn_abort(const spava_problem_t* prob, const void* Q, const void* K,
+                                      const void* V, const void* Kp, const void* Vp, void* O, float* lse,
+                                      float* O_part, float* lse_part, int32_t skip_k_tile,
+                                      uint64_t limit_ns, spava_stream_t stream);
+
 /* Human-readable name of a status code (static string). */
 const char* spava_status_string(spava_status_t status);
 

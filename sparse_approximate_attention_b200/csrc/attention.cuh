@@ -59,6 +59,12 @@ struct AttnParams {
   // the passing buffer and the merge counters are read only after
   // griddepcontrol.wait.
   int32_t pdl_wait;
+  // Bounded waits: every wait gives up after wait_limit_ns (4 s in the
+  // layer).  skip_k_tile >= 0 (a test hook, -1 in the layer): the producer
+  // does not load that key tile, so the waits for it run out and the CTA
+  // takes its abort path.
+  int32_t skip_k_tile;
+  uint64_t wait_limit_ns;
   Region regions[kMaxRegions];
   uint32_t items[kMaxItems];   // (region << 20) | pair of 128-row tiles
 };
@@ -257,7 +263,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1)
       for (int j = 0; j <= ntk; ++j) {
         if (j < ntk) {
           const int st = j % KS;
-          if (j >= KS && !mbar_wait(BAR_KE(st), ((j / KS) - 1) & 1, abort_flag)) break;
+          if (j >= KS && !mbar_wait(BAR_KE(st), ((j / KS) - 1) & 1, abort_flag, p.wait_limit_ns)) break;
           const Seg& sg = R.seg[ik.s];
           if (sg.src == kSrcPass && !waited) {   // the passing buffer is written by the preceding grid
             grid_dependency_wait();
@@ -265,15 +271,17 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1)
           }
           const CUtensorMap* tk = sg.src == kSrcMain ? &p.tm_k : &p.tm_kp;
           const int krow = sg.start + ik.kt * kBN;
-          mbar_arrive_expect_tx(BAR_KF(st), C::kTileBytes);
-          for (int sl = 0; sl < C::kSlabs; ++sl)
-            tma_load_3d(sK + st * C::kTileBytes + sl * C::kSlabBytes, tk, BAR_KF(st), sl * 64, kv, krow);
+          if (j != p.skip_k_tile) {
+            mbar_arrive_expect_tx(BAR_KF(st), C::kTileBytes);
+            for (int sl = 0; sl < C::kSlabs; ++sl)
+              tma_load_3d(sK + st * C::kTileBytes + sl * C::kSlabBytes, tk, BAR_KF(st), sl * 64, kv, krow);
+          }
           k_issued = j + 1;
           iter_next(ik);
         }
         if (j >= 1) {
           const int i = j - 1, st = i % VS;
-          if (i >= VS && !mbar_wait(BAR_VE(st), ((i / VS) - 1) & 1, abort_flag)) break;
+          if (i >= VS && !mbar_wait(BAR_VE(st), ((i / VS) - 1) & 1, abort_flag, p.wait_limit_ns)) break;
           const Seg& sg = R.seg[iv.s];
           const CUtensorMap* tv = sg.src == kSrcMain ? &p.tm_v : &p.tm_vp;
           const int krow = sg.start + iv.kt * kBN;
@@ -285,9 +293,11 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1)
         }
       }
       if (*abort_flag) {   // let copies already in flight land before the CTA exits
-        mbar_wait_drain(BAR_Q, 0);
-        for (int j = max(0, k_issued - KS); j < k_issued; ++j) mbar_wait_drain(BAR_KF(j % KS), (j / KS) & 1);
-        for (int j = max(0, v_issued - VS); j < v_issued; ++j) mbar_wait_drain(BAR_VF(j % VS), (j / VS) & 1);
+        const uint64_t dl = p.wait_limit_ns / 4;
+        mbar_wait_drain(BAR_Q, 0, dl);
+        for (int j = max(0, k_issued - KS); j < k_issued; ++j)
+          if (j != p.skip_k_tile) mbar_wait_drain(BAR_KF(j % KS), (j / KS) & 1, dl);
+        for (int j = max(0, v_issued - VS); j < v_issued; ++j) mbar_wait_drain(BAR_VF(j % VS), (j / VS) & 1, dl);
       }
     }
   } else if (warp == 1) {
@@ -307,7 +317,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1)
       const uint32_t k_lo = (sK >> 4) | (1u << 16);
       const uint32_t v_lo = (sV >> 4) | ((static_cast<uint32_t>(C::kSlabBytes) >> 4) << 16);
       auto wait = [&](uint32_t bar, uint32_t parity) {
-        return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+        return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, p.wait_limit_ns));
       };
       // S_t = Q_t K_j^T into TMEM buffer t
       auto issue_s = [&](int t, int j) {
@@ -363,7 +373,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1)
       }
       if (ok && nt1 > 0) issue_pv(1, nt1 - 1, true, true);
       mma_commit_warp(BAR_FIN);   // every MMA issued above has finished once this lands
-      mbar_wait_drain(BAR_FIN, 0);
+      mbar_wait_drain(BAR_FIN, 0, p.wait_limit_ns / 4);
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax
@@ -394,7 +404,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1)
     }
     TileIter it = iter_begin();
     for (int j = 0; j < nt; ++j) {
-      ok = __all_sync(0xffffffffu, mbar_wait(BAR_SF(qt), j & 1, abort_flag));
+      ok = __all_sync(0xffffffffu, mbar_wait(BAR_SF(qt), j & 1, abort_flag, p.wait_limit_ns));
       if (!ok) break;
       tc_fence_after();
       float2 x[kBN / 2];
@@ -476,7 +486,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::kThreads, 1)
       iter_next(it);
     }
     if (ok && nt > 0) {   // BAR_OD(t) completes once, after the last O_t += P V
-      ok = __all_sync(0xffffffffu, mbar_wait(BAR_OD(qt), 0, abort_flag));
+      ok = __all_sync(0xffffffffu, mbar_wait(BAR_OD(qt), 0, abort_flag, p.wait_limit_ns));
     }
     if (ok && nt > 0) {
       tc_fence_after();

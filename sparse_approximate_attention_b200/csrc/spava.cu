@@ -430,7 +430,8 @@ spava_status_t run_compress(const Plan& P, const void* Q, const void* K, const v
 // counters.
 spava_status_t run_attn(const Plan& P, const void* Q, const void* K, const void* V, const void* Kp,
                         const void* Vp, void* O, float* lse, float* O_part, float* lse_part,
-                        int32_t* merge_count, bool dependent, cudaStream_t st, int tag = 0) {
+                        int32_t* merge_count, bool dependent, cudaStream_t st, int tag = 0,
+                        int skip_k_tile = -1, uint64_t wait_limit_ns = kWaitLimitNs) {
   if (!Q || !K || !V || !O || !lse || !O_part || !lse_part) return SPAVA_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(O_part))
     return SPAVA_ERR_INVALID_ARG;
@@ -449,6 +450,8 @@ spava_status_t run_attn(const Plan& P, const void* Q, const void* K, const void*
   prm.lse_part = lse_part;
   prm.merge_count = merge_count;
   prm.pdl_wait = dependent ? 1 : 0;
+  prm.skip_k_tile = skip_k_tile;
+  prm.wait_limit_ns = wait_limit_ns;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(e->grid));
   cfg.stream = st;
@@ -731,6 +734,18 @@ spava_status_t spava_device_error(uint32_t* code) {
   if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess) return SPAVA_ERR_CUDA;
   *code = v;
   return SPAVA_OK;
+}
+
+spava_status_t spava_debug_attn_abort(const spava_problem_t* prob, const void* Q, const void* K, const void* V,
+                                      const void* Kp, const void* Vp, void* O, float* lse, float* O_part,
+                                      float* lse_part, int32_t skip_k_tile, uint64_t limit_ns,
+                                      spava_stream_t stream) {
+  Plan P;
+  spava_status_t s = make_plan(prob, &P);
+  if (s != SPAVA_OK) return s;
+  if (skip_k_tile < 0 || limit_ns == 0 || limit_ns > kWaitLimitNs) return SPAVA_ERR_INVALID_ARG;
+  return run_attn(P, Q, K, V, Kp, Vp, O, lse, O_part, lse_part, nullptr, false,
+                  reinterpret_cast<cudaStream_t>(stream), 0, skip_k_tile, limit_ns);
 }
 
 spava_status_t spava_debug_wait_timeout(int64_t* out, uint64_t limit_ns, spava_stream_t stream) {

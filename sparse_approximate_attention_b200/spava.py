@@ -60,6 +60,7 @@ _SIGS = {
     "spava_device_error": [ctypes.POINTER(ctypes.c_uint32)],
     "spava_layer_fwd_noalloc": [_PP, _VP, _VP, _VP, _VP, _VP, _VP],
     "spava_debug_wait_timeout": [_VP, ctypes.c_uint64, _VP],
+    "spava_debug_attn_abort": [_PP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_int32, ctypes.c_uint64, _VP],
 }
 
 
@@ -314,3 +315,17 @@ def debug_wait_timeout(limit_ns: int, stream=None):
     out = torch.zeros(4, dtype=torch.int64, device="cuda")
     _check("spava_debug_wait_timeout", lib().spava_debug_wait_timeout(_ptr(out), int(limit_ns), _stream(stream)))
     return tuple(int(v) for v in out.cpu().tolist())
+
+
+def debug_attn_abort(p: Problem, Q, K, V, Kp, Vp, skip_k_tile: int, limit_ns: int, stream=None):
+    """Test hook: the attention launch with key tile skip_k_tile left
+    unloaded and every wait limited to limit_ns (its outputs are invalid)."""
+    sh = _shapes(p)[1]
+    dev = Q.device
+    O = torch.empty(sh["O"], dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(sh["lse"], dtype=torch.float32, device=dev)
+    O_part = torch.empty(sh["O_part"], dtype=torch.float32, device=dev)
+    lse_part = torch.empty(sh["lse_part"], dtype=torch.float32, device=dev)
+    _check("spava_debug_attn_abort", lib().spava_debug_attn_abort(
+        p.ref, _ptr(Q), _ptr(K), _ptr(V), _ptr(Kp), _ptr(Vp), _ptr(O), _ptr(lse), _ptr(O_part), _ptr(lse_part),
+        int(skip_k_tile), int(limit_ns), _stream(stream)))

@@ -389,3 +389,26 @@ def test_bounded_wait_gives_up_reports_and_leaves_the_context_usable():
     _no_device_error()
     assert max_err(to_np(O).astype(np.float64), ref["O"]) <= O_TOL
     assert max_err(to_np(lse), ref["lse"]) <= LSE_TOL
+
+
+@pytest.mark.parametrize("name", ["frames_multi", "pair_lq1_d64"])
+def test_attention_abort_path_drains_and_leaves_the_context_usable(name):
+    """The attention kernel's own abort path: with key tile 1 left unloaded
+    and every wait limited to 50 ms, the CTAs that reach the tile give up,
+    drain what is in flight, free TMEM and set the device error word; the
+    same attention then runs correctly on the same context."""
+    wl, lay, inp, ref = _case(name)
+    p = spava.Problem.from_workload(wl)
+    d = _dev(inp)
+    Kp, Vp = _oracle_passing_dev(lay, inp, ref, wl.num_kv_heads, wl.head_dim)
+    _no_device_error()
+    spava.debug_attn_abort(p, d["Q"], d["K"], d["V"], Kp, Vp, skip_k_tile=1, limit_ns=50_000_000)
+    torch.cuda.synchronize()
+    assert spava.device_error() == 1
+    O, lse, O_part, lse_part = spava.attn_fwd(p, d["Q"], d["K"], d["V"], Kp, Vp)
+    torch.cuda.synchronize()
+    _no_device_error()
+    qs = lay.query_start
+    assert max_err(to_np(O)[:qs], ref["O"][:qs]) <= O_TOL
+    assert max_err(to_np(lse)[:, :qs], ref["lse"][:, :qs]) <= LSE_TOL
+    assert max_err(to_np(O_part), ref["o_part"]) <= O_TOL
