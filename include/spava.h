@@ -167,9 +167,10 @@ spava_status_t spava_gather_passing(const spava_problem_t* prob, const void* K,
 
 /* Steps 1-3 fused in one launch: the same qsum, scores, idx, Kp and Vp as
  * spava_score + spava_select_topk + spava_gather_passing ([SC] Fig. 5 caption:
- * importance estimation, then the essential KVs).  One cluster of 8 CTAs per
- * (block, KV head) streams K^(h) once, selects in shared memory and copies the
- * kept rows.  Every block length must be <= 24576 (SPAVA_ERR_UNSUPPORTED
+ * importance estimation, then the essential KVs).  One cluster of CTAs per
+ * (block, KV head) -- 8, or 4 when 8-CTA clusters would not fit the GPU in one
+ * wave -- streams K^(h) once, selects in shared memory and copies the kept
+ * rows.  Every block length must be <= 24576 (SPAVA_ERR_UNSUPPORTED
  * otherwise; the separate stage calls have no such limit).  With lp = 0 it
  * does nothing.  With a partial host_mask only the selected blocks are
  * compressed: their scores, idx and Kp/Vp rows (at their offsets off_h of the
