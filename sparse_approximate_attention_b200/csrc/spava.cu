@@ -475,8 +475,9 @@ spava_status_t run_attn(const Plan& P, const void* Q, const void* K, const void*
 spava_status_t run_merge(const Plan& P, const float* O_part, const float* lse_part, void* O, float* lse,
                          cudaStream_t st) {
   if (!O_part || !lse_part || !O || !lse || !aligned16(O_part) || !aligned16(O)) return SPAVA_ERR_INVALID_ARG;
-  const int64_t total = static_cast<int64_t>(P.lq) * P.Hq * (P.d / 4);
-  const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((total + 255) / 256, sm_count() * 8));
+  if (P.V > 32) return SPAVA_ERR_UNSUPPORTED;   // one lane per partial
+  const int64_t pairs = static_cast<int64_t>(P.lq) * P.Hq;   // one warp per (row, head), 8 per block
+  const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((pairs + 7) / 8, sm_count() * 16));
   auto* o = static_cast<__nv_bfloat16*>(O);
   if (P.d == 128)
     merge_kernel<128><<<static_cast<unsigned>(blocks), 256, 0, st>>>(O_part, lse_part, o, lse, P.V, P.lq, P.Hq,
