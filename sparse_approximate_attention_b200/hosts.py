@@ -11,7 +11,8 @@ their log-sum-exp ("Axiom & Free-Parameter Ledger": the merge is exact).
 
 One process per GPU (torch.distributed; NCCL between GPUs, gloo on CPU).  The
 physical hosts are dealt to the ranks round-robin (p % world == rank), so a
-rank holds whole ZigZag pairs.  Per layer every rank
+rank holds whole ZigZag pairs; with more ranks than physical hosts the extra
+ranks hold none and only take part in the collectives.  Per layer every rank
   1. compresses its own context blocks (spava_compress with its host mask):
      their scores, indices and passing rows, at their offsets of the full
      passing buffer;
@@ -145,6 +146,8 @@ class HostShardedLayer:
                  dtypes=(torch.bfloat16, torch.float32)):
         self.p, self.world, self.rank = p, world, rank
         self.mask = host_mask(p.num_hosts, world, rank)
+        # a rank without hosts (world > H) computes nothing: host_mask 0 would mean "every host"
+        self.idle = self.mask == 0
         self.q = p.with_hosts(self.mask)
         self.ex = HostExchange(p, world, rank, group)
         self.k = kernels if kernels is not None else spava
@@ -163,11 +166,12 @@ class HostShardedLayer:
     def forward(self, Q, K, V, O, lse, stream=None) -> None:
         """O and lse: this rank's rows (its hosts' context rows, the anchor rows
         on the rank of host 0) and, on every rank, the query rows."""
-        if self.p.lp > 0:
+        if self.p.lp > 0 and not self.idle:
             self.k.compress(self.q, Q, K, V, self.qsum, self.scores, self.idx, self.Kp, self.Vp, stream=stream)
         self.ex.exchange_passing(self.Kp, self.Vp)
-        self.k.attn_fwd(self.q, Q, K, V, self.Kp if self.p.lp else None, self.Vp if self.p.lp else None,
-                        O, lse, self.O_part, self.lse_part, stream=stream)
+        if not self.idle:
+            self.k.attn_fwd(self.q, Q, K, V, self.Kp if self.p.lp else None, self.Vp if self.p.lp else None,
+                            O, lse, self.O_part, self.lse_part, stream=stream)
         self.ex.exchange_partials(self.O_part, self.lse_part)
         self.k.lse_merge(self.p, self.O_part, self.lse_part, O, lse, stream=stream)
 

@@ -130,8 +130,10 @@ def _worker(rank, world, port, out):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("world", [2, 3, 5])
 def test_gloo_ranks_exchange_passing_rows_and_query_partials(world):
+    """world 5 > H = 4: rank 4 holds no host, computes nothing and still takes
+    part in both all-gathers."""
     out = mp.Manager().dict()
     mp.spawn(_worker, args=(world, _free_port(), out), nprocs=world, join=True)
     lay = oracle.make_layout(**CASE)
