@@ -7,9 +7,9 @@ TFLOP/s against the measured bf16 tensor-core peak.
                     [--impl reference]
 
 One step = one spava_layer_fwd call over one synthetic input set: the
-compression launch (query-block sum, scores, top-lp, passing gather), then
-the attention launch, which also merges the query partials and starts while
-the compression runs.  The default workload is the 256K-token long-video
+query-block sum, the compression launch (scores, top-lp, passing gather),
+then the attention launch, which also merges the query partials; each starts
+while the one before it runs (programmatic dependent launch).  The default workload is the 256K-token long-video
 stress case with lp = 4096, the largest that fits one GPU.  Timed on the
 device with CUDA events; inputs rotate over three resident sets, each larger
 than L2.  The attention, compression and stage-merge kernels are then timed
@@ -330,7 +330,8 @@ def run_gpu(args, wl):
             x = sets[k % 3]
             sharded.forward(x["Q"], x["K"], x["V"], O, lse, stream=stream)
 
-        launches_per_step = 3 if lp > 0 else 2   # compression, attention, merge (collectives are NCCL's)
+        # query sum + compression, attention, merge (collectives are NCCL's)
+        launches_per_step = 4 if lp > 0 else 2
     else:
         q = p
 
@@ -338,7 +339,8 @@ def run_gpu(args, wl):
             x = sets[k % 3]
             spava.layer_fwd(p, x["Q"], x["K"], x["V"], O, lse, ws, stream=stream)
 
-        launches_per_step = 2   # compression (or the zeroing of the merge counters when lp = 0) + attention
+        # query sum + compression, then attention (lp = 0: a memset of the merge counters + attention)
+        launches_per_step = 3 if lp > 0 else 1
 
     for i in range(args.warmup):
         layer(i)
@@ -521,8 +523,8 @@ def report(args, wl, sz, world, n, ms_per_step, elapsed_ms, value, stage_ms, att
         "stages": stage_info,
         "layer": ("per rank: spava_compress and spava_attn_fwd with the rank's host mask, all-gathers of "
                   "passing rows and query partials, spava_lse_merge") if hosts_mode else
-                 ("spava_layer_fwd: compression launch, then attention with the query-partial merge "
-                  "(programmatic dependent launch)"),
+                 ("spava_layer_fwd: query-sum launch, compression cluster launch, then attention with the "
+                  "query-partial merge (each a programmatic dependent launch of the one before)"),
         "e2e": None if e2e_ms is None else {
             "value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3),

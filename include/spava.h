@@ -165,16 +165,20 @@ spava_status_t spava_gather_passing(const spava_problem_t* prob, const void* K,
                                     const void* V, const int32_t* idx,
                                     void* Kp, void* Vp, spava_stream_t stream);
 
-/* Steps 1-3 fused in one launch: the same qsum, scores, idx, Kp and Vp as
+/* Steps 1-3 fused in two launches: the same qsum, scores, idx, Kp and Vp as
  * spava_score + spava_select_topk + spava_gather_passing ([SC] Fig. 5 caption:
- * importance estimation, then the essential KVs).  One cluster of CTAs per
+ * importance estimation, then the essential KVs).  The query-block sum (the
+ * scoring stage's own kernel, so both calls see the same qsum bits), then,
+ * started at once as its programmatic dependent, one cluster of CTAs per
  * (block, KV head) -- 8, or 4 when 8-CTA clusters would not fit the GPU in one
- * wave -- streams K^(h) once, selects in shared memory and copies the kept
- * rows.  Every block length must be <= 24576 (SPAVA_ERR_UNSUPPORTED
- * otherwise; the separate stage calls have no such limit).  With lp = 0 it
- * does nothing.  With a partial host_mask only the selected blocks are
- * compressed: their scores, idx and Kp/Vp rows (at their offsets off_h of the
- * full buffer) are written, nothing else. */
+ * wave -- streams K^(h) once (each CTA one slice), selects across the cluster
+ * by exchanging radix counts in distributed shared memory and copies the kept
+ * rows, an equal share per CTA.  Every block length must be <= 24576
+ * (SPAVA_ERR_UNSUPPORTED otherwise; the separate stage calls have no such
+ * limit).  With lp = 0 it does nothing.  With a partial host_mask only the
+ * selected blocks are compressed: their scores, idx and Kp/Vp rows (at their
+ * offsets off_h of the full buffer) are written, and qsum if any block is
+ * selected; nothing else. */
 spava_status_t spava_compress(const spava_problem_t* prob, const void* Q,
                               const void* K, const void* V, float* qsum,
                               float* scores, int32_t* idx, void* Kp, void* Vp,
@@ -206,7 +210,8 @@ spava_status_t spava_lse_merge(const spava_problem_t* prob, const float* O_part,
 /* The whole layer: steps 1-5 in order on `stream`, with every intermediate
  * carved from `workspace` (device memory, >= spava_workspace_size bytes,
  * 256-byte aligned).  Outputs O [n, Hq, d] bf16 and lse [Hq, n] fp32.
- * Two launches: the one-launch compression (steps 1-3), then attention with
+ * Three launches: the compression of steps 1-3 (query sum, then scores,
+ * selection and gather in one cluster launch), then attention with
  * the merge of step 5 in the same launch (the last of the V partial CTAs of
  * a query tile pair merges it; [SC] Fig. 5 caption: the passing-block
  * exchange and the merge overlap the attention).  The attention launch may

@@ -20,54 +20,77 @@ namespace cg = cooperative_groups;
 // ---------------------------------------------------------------------------
 // qsum[kv][c] = scale * sum over query rows i and heads g of KV head kv of
 // Q[qs+i, g, c].  One cluster of kQsumSplit CTAs per KV head: each CTA sums a
-// slice of the (row, head) pairs, then CTA 0 adds the slices in a fixed order
-// through distributed shared memory (deterministic, one launch).
+// slice of the (row, head) pairs (kQsumUnroll 16-byte loads per thread in
+// flight), pushes its slice sum into CTA 0 through distributed shared
+// memory, and CTA 0 adds the slices in rank order (deterministic, one
+// launch).  The order of every addition is fixed by the problem's sizes
+// alone, so the scoring stage and the fused compression, which both start
+// with this kernel, see the same qsum bits.
 // ---------------------------------------------------------------------------
 constexpr int kQsumSplit = 8;
-constexpr int kQsumThreads = 256;
+constexpr int kQsumThreads = 512;
+constexpr int kQsumUnroll = 8;
 
 template <int D>
-__global__ void __cluster_dims__(kQsumSplit, 1, 1) __launch_bounds__(kQsumThreads)
+__global__ void __cluster_dims__(kQsumSplit, 1, 1) __launch_bounds__(kQsumThreads, 1)
     qsum_kernel(const __nv_bfloat16* __restrict__ Q, float* __restrict__ qsum, int64_t qs, int lq,
                 int Hq, int G, float scale) {
   constexpr int kParts = D / 8;                    // 16-byte chunks per row
-  constexpr int kLanesRows = kQsumThreads / kParts;
-  __shared__ float part[kLanesRows][D];
-  __shared__ float slice[D];
+  constexpr int kRows = kQsumThreads / kParts;     // rows per pass of the CTA
+  constexpr int kWarps = kQsumThreads / 32;
+  __shared__ float part[kWarps][D];
+  __shared__ float gathered[kQsumSplit][D];
+  // A kernel launched after this one as its programmatic dependent (the fused
+  // compression) may start now; it waits for this grid before reading qsum.
+  if (threadIdx.x == 0) grid_dependents_launch();
   cg::cluster_group cluster = cg::this_cluster();
   const int kv = blockIdx.y;
   const int rank = static_cast<int>(cluster.block_rank());
   const int total = lq * G;
   const int r0 = static_cast<int>((static_cast<int64_t>(total) * rank) / kQsumSplit);
   const int r1 = static_cast<int>((static_cast<int64_t>(total) * (rank + 1)) / kQsumSplit);
-  const int pc = threadIdx.x % kParts, lr = threadIdx.x / kParts;
+  const int tid = threadIdx.x, pc = tid % kParts, lr = tid / kParts;
   float acc[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-  for (int rr = r0 + lr; rr < r1; rr += kLanesRows) {
-    const int i = rr / G, g = kv * G + rr % G;
-    const uint4 raw = *reinterpret_cast<const uint4*>(Q + ((qs + i) * Hq + g) * D + pc * 8);
-    const __nv_bfloat16* v = reinterpret_cast<const __nv_bfloat16*>(&raw);
+  for (int rb = r0 + lr; rb < r1; rb += kQsumUnroll * kRows) {
+    uint4 raw[kQsumUnroll];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] += __bfloat162float(v[e]);
+    for (int u = 0; u < kQsumUnroll; ++u) {
+      const int rr = rb + u * kRows;
+      const int i = rr / G, g = kv * G + rr % G;
+      raw[u] = rr < r1 ? *reinterpret_cast<const uint4*>(Q + ((qs + i) * Hq + g) * D + pc * 8)
+                       : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < kQsumUnroll; ++u) {
+      const __nv_bfloat16* v = reinterpret_cast<const __nv_bfloat16*>(&raw[u]);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] += __bfloat162float(v[e]);
+    }
   }
+  // lanes l and l ^ 16 hold the same column chunk (for D = 128): add them
 #pragma unroll
-  for (int e = 0; e < 8; ++e) part[lr][pc * 8 + e] = acc[e];
+  for (int off = kParts; off < 32; off <<= 1)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
+  if ((tid & 31) < kParts)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) part[tid >> 5][pc * 8 + e] = acc[e];
   __syncthreads();
-  for (int c = threadIdx.x; c < D; c += kQsumThreads) {
+  for (int c = tid; c < D; c += kQsumThreads) {
     float s = 0.f;
-    for (int j = 0; j < kLanesRows; ++j) s += part[j][c];
-    slice[c] = s;
+    for (int w = 0; w < kWarps; ++w) s += part[w][c];
+    cluster.map_shared_rank(&gathered[rank][0], 0)[c] = s;
   }
-  cluster.sync();
+  cluster.sync();   // CTA 0 holds every slice; no CTA touches another's memory after this
   if (rank == 0) {
-    for (int c = threadIdx.x; c < D; c += kQsumThreads) {
+    for (int c = tid; c < D; c += kQsumThreads) {
       float s = 0.f;
-      for (int j = 0; j < kQsumSplit; ++j) s += cluster.map_shared_rank(slice, j)[c];
+      for (int r = 0; r < kQsumSplit; ++r) s += gathered[r][c];
       qsum[kv * D + c] = s * scale;
     }
   }
-  cluster.sync();
 }
 
 // ---------------------------------------------------------------------------

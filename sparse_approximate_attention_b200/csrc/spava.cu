@@ -71,7 +71,12 @@ struct DeviceSetup {
   spava_status_t status = SPAVA_OK;
   int sm_count = 148;
   int smem_per_sm = 228 * 1024;      // shared memory of one SM
+  int smem_optin = 227 * 1024;       // largest dynamic + static shared memory of one CTA
+  int smem_reserved = 1024;          // shared memory the system reserves per CTA
   int compress_static[2] = {0, 0};   // static shared memory of compress_kernel<64>, <128>
+  // cudaOccupancyMaxActiveClusters of compress_kernel, by (d, nc, dynamic smem)
+  struct ClusterFit { int d, nc, smem, clusters; };
+  std::vector<ClusterFit> compress_fit;
 };
 std::mutex g_setup_mu;
 DeviceSetup g_setup[kMaxDevices];
@@ -104,6 +109,10 @@ spava_status_t device_setup(const DeviceSetup** out) {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0) s.sm_count = n;
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) == cudaSuccess && n > 0)
       s.smem_per_sm = n;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) == cudaSuccess && n > 0)
+      s.smem_optin = n;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrReservedSharedMemoryPerBlock, dev) == cudaSuccess && n >= 0)
+      s.smem_reserved = n;
     spava_status_t st = setup_attn<128>();
     if (st == SPAVA_OK) st = setup_attn<64>();
     if (st == SPAVA_OK &&
@@ -112,18 +121,19 @@ spava_status_t device_setup(const DeviceSetup** out) {
          cudaFuncSetAttribute(colsum_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               ColsumCfg<64>::kSmemBytes) != cudaSuccess))
       st = SPAVA_ERR_CUDA;
-    const int csmem = compress_smem_bytes(kCompressMaxBlock, kCompressMinCtas);
-    if (st == SPAVA_OK &&
-        (cudaFuncSetAttribute(compress_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, csmem) !=
-             cudaSuccess ||
-         cudaFuncSetAttribute(compress_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, csmem) !=
-             cudaSuccess))
-      st = SPAVA_ERR_CUDA;
+    // compress_kernel may ask for up to the whole per-CTA limit (a launch that
+    // wants one CTA per SM pads its request)
     cudaFuncAttributes fa;
     if (st == SPAVA_OK && cudaFuncGetAttributes(&fa, compress_kernel<64>) == cudaSuccess)
       s.compress_static[0] = static_cast<int>(fa.sharedSizeBytes);
     if (st == SPAVA_OK && cudaFuncGetAttributes(&fa, compress_kernel<128>) == cudaSuccess)
       s.compress_static[1] = static_cast<int>(fa.sharedSizeBytes);
+    if (st == SPAVA_OK &&
+        (cudaFuncSetAttribute(compress_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              s.smem_optin - s.compress_static[0]) != cudaSuccess ||
+         cudaFuncSetAttribute(compress_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              s.smem_optin - s.compress_static[1]) != cudaSuccess))
+      st = SPAVA_ERR_CUDA;
     s.status = st;
     s.done = true;
   }
@@ -337,20 +347,55 @@ spava_status_t run_gather(const Plan& P, const void* K, const void* V, const int
   return last_launch();
 }
 
+// Clusters of nc compress_kernel CTAs with `smem` dynamic bytes that can be
+// resident at once (0 when the query fails); cached per device.
+int compress_clusters(const DeviceSetup* ds, int d, int nc, int smem) {
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  auto& fit = const_cast<DeviceSetup*>(ds)->compress_fit;
+  for (const auto& f : fit)
+    if (f.d == d && f.nc == nc && f.smem == smem) return f.clusters;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(nc);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(static_cast<unsigned>(nc), 1, 1);
+  cfg.blockDim = dim3(kCompressThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  const cudaError_t e = d == 128 ? cudaOccupancyMaxActiveClusters(&n, compress_kernel<128>, &cfg)
+                                 : cudaOccupancyMaxActiveClusters(&n, compress_kernel<64>, &cfg);
+  if (e != cudaSuccess) {
+    cudaGetLastError();   // a failed query is not a launch error
+    n = 0;
+  }
+  fit.push_back({d, nc, smem, n});
+  return n;
+}
+
 bool compress_fits(const Plan& P) {
   for (int h = 0; h < P.V - 1; ++h)
     if (P.L[h] > kCompressMaxBlock) return false;
   return true;
 }
 
-// Steps 1-3 in one launch: one cluster of nc CTAs per (block, KV head).
-// merge_count (may be null): the following attention launch's merge
-// counters, zeroed by this launch.
+// Steps 1-3 in two launches: the query-block sum (qsum_kernel, the same
+// kernel as the scoring stage's), then one cluster of nc CTAs per (block, KV
+// head), launched as the sum's programmatic dependent: it starts its K stream
+// at once and waits for the sum before its first score.  merge_count (may be
+// null): the following attention launch's merge counters, zeroed by the
+// second launch.
 //
-// nc: 8 if the grid of 8-CTA clusters fits the GPU in one wave (two CTAs per
-// SM when the shared memory allows it), else 4, so that as many CTAs as
-// possible stream their slice of K at the same time.  The K stream and the
-// gather shrink with nc, the key broadcast and the local select do not.
+// The launch shape is the first of: 8-CTA clusters with one CTA per SM,
+// 4-CTA clusters with one CTA per SM, 8-CTA clusters packed two per SM, 4-CTA
+// clusters packed, that fits the GPU in one wave (cudaOccupancyMaxActiveClusters,
+// which knows how clusters fill the GPCs); 4-CTA clusters packed when none
+// does.  One CTA per SM is forced by padding the shared-memory request: two
+// CTAs on one SM share its load bandwidth and set the launch's span.
 spava_status_t run_compress(const Plan& P, const void* Q, const void* K, const void* V, float* qsum,
                             float* scores, int32_t* idx, void* Kp, void* Vp, int32_t* merge_count,
                             cudaStream_t st) {
@@ -370,15 +415,10 @@ spava_status_t run_compress(const Plan& P, const void* Q, const void* K, const v
     cp.k[h] = P.lpe[h];
   }
   for (int h = 0; h <= P.V; ++h) cp.poff[h] = P.poff[h];
-  cp.Hq = P.Hq;
   cp.Hkv = P.Hkv;
-  cp.G = P.G;
-  cp.lq = P.lq;
   cp.lp = P.lp;
-  cp.qs = P.qs;
   cp.la = P.la;
   cp.score_cols = P.score_cols;
-  cp.scale = P.scale;
   cp.merge_count = merge_count;
   cp.n_merge = merge_count ? P.n_merge : 0;
   if (P.ncblk == 0) return SPAVA_OK;   // a host mask that selects no compressed block
@@ -387,37 +427,50 @@ spava_status_t run_compress(const Plan& P, const void* Q, const void* K, const v
     cp.lmax = std::max(cp.lmax, P.L[P.cblk[i]]);
   }
   const int pairs = P.ncblk * P.Hkv;
-  int nc = kCompressMinCtas;
-  for (int c = kCompressMaxCtas; c > kCompressMinCtas; c /= 2) {
-    // a CTA's shared memory: dynamic + static + the 1 KB the system reserves per CTA
-    const int cta_bytes = compress_smem_bytes(cp.lmax, c) + ds->compress_static[P.d == 128 ? 1 : 0] + 1024;
-    const int per_sm = std::min(2, std::max(1, ds->smem_per_sm / cta_bytes));
-    if (static_cast<int64_t>(pairs) * c <= static_cast<int64_t>(per_sm) * ds->sm_count) {
-      nc = c;
+  const int stat = ds->compress_static[P.d == 128 ? 1 : 0];
+  // dynamic bytes above which two CTAs (dynamic + static + what the system
+  // reserves per CTA) no longer fit one SM
+  const int spread = (ds->smem_per_sm / 2 - stat - ds->smem_reserved + 16) / 16 * 16;
+  int nc = kCompressMinCtas, smem = compress_smem_bytes(cp.lmax, kCompressMinCtas);
+  const struct { int nc; bool spread; } shapes[4] = {{8, true}, {4, true}, {8, false}, {4, false}};
+  for (const auto& sh : shapes) {
+    int b = compress_smem_bytes(cp.lmax, sh.nc);
+    if (sh.spread) b = std::max(b, spread);
+    if (b + stat > ds->smem_optin) continue;
+    if (compress_clusters(ds, P.d, sh.nc, b) >= pairs) {
+      nc = sh.nc;
+      smem = b;
       break;
     }
   }
-  const int smem = compress_smem_bytes(cp.lmax, nc);
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = static_cast<unsigned>(nc);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.gridDim = dim3(static_cast<unsigned>(nc), static_cast<unsigned>(P.ncblk), static_cast<unsigned>(P.Hkv));
-  cfg.blockDim = dim3(kCompressThreads);
-  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
-  cfg.stream = st;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
   const auto* q = static_cast<const __nv_bfloat16*>(Q);
   const auto* k = static_cast<const __nv_bfloat16*>(K);
   const auto* v = static_cast<const __nv_bfloat16*>(V);
   auto* kp = static_cast<__nv_bfloat16*>(Kp);
   auto* vp = static_cast<__nv_bfloat16*>(Vp);
+  const dim3 qgrid(kQsumSplit, P.Hkv);
+  if (P.d == 128)
+    qsum_kernel<128><<<qgrid, kQsumThreads, 0, st>>>(q, qsum, P.qs, P.lq, P.Hq, P.G, P.scale);
+  else
+    qsum_kernel<64><<<qgrid, kQsumThreads, 0, st>>>(q, qsum, P.qs, P.lq, P.Hq, P.G, P.scale);
+  if (last_launch() != SPAVA_OK) return SPAVA_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(nc);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3(static_cast<unsigned>(nc), static_cast<unsigned>(P.ncblk), static_cast<unsigned>(P.Hkv));
+  cfg.blockDim = dim3(kCompressThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
   const cudaError_t e = P.d == 128
-                            ? cudaLaunchKernelEx(&cfg, compress_kernel<128>, q, k, v, qsum, scores, idx, kp, vp, cp)
-                            : cudaLaunchKernelEx(&cfg, compress_kernel<64>, q, k, v, qsum, scores, idx, kp, vp, cp);
+                            ? cudaLaunchKernelEx(&cfg, compress_kernel<128>, k, v, qsum, scores, idx, kp, vp, cp)
+                            : cudaLaunchKernelEx(&cfg, compress_kernel<64>, k, v, qsum, scores, idx, kp, vp, cp);
   if (e != cudaSuccess) return SPAVA_ERR_CUDA;
   return last_launch();
 }
@@ -541,7 +594,7 @@ spava_status_t run_score_variant(const Plan& P, const void* Q, const void* K, fl
 }
 
 // The whole layer with its intermediates carved from `ws` (P.ws_total bytes,
-// 256-byte aligned): compression (one launch, or the three stage kernels for
+// 256-byte aligned): compression (qsum + one cluster launch, or the stage kernels for
 // blocks too long for it), then attention with the query-partial merge in
 // the same launch, started as a programmatic dependent of the compression.
 // The work list is built (and checked) before anything is launched.
@@ -571,7 +624,7 @@ spava_status_t run_layer(const Plan& P, uint8_t* ws, const void* Q, const void* 
     if ((s = run_gather(P, K, V, idx, Kp, Vp, st)) != SPAVA_OK) return s;
     if (cudaMemsetAsync(count, 0, sizeof(int32_t) * static_cast<size_t>(P.n_merge), st) != cudaSuccess)
       return SPAVA_ERR_CUDA;
-  } else if (P.lp > 0 && compress_fits(P)) {   // steps 1-3 in one launch; it also zeroes the merge counters
+  } else if (P.lp > 0 && compress_fits(P)) {   // steps 1-3 in two launches; the second zeroes the merge counters
     if ((s = run_compress(P, Q, K, V, qsum, scores, idx, Kp, Vp, count, st)) != SPAVA_OK) return s;
     dependent = true;
   } else {

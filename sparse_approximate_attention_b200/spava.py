@@ -211,7 +211,8 @@ def gather_passing(p: Problem, K, V, idx, Kp=None, Vp=None, stream=None):
 
 
 def compress(p: Problem, Q, K, V, qsum=None, scores=None, idx=None, Kp=None, Vp=None, stream=None):
-    """Steps 1-3 in one launch (scores, top-lp indices, passing buffer)."""
+    """Steps 1-3 fused (query sum, then scores, top-lp indices and passing
+    buffer in one cluster launch)."""
     sz, sh = _shapes(p)
     for t, nm in ((Q, "Q"), (K, "K"), (V, "V")):
         _need(t, torch.bfloat16, sh[nm], nm)

@@ -127,7 +127,7 @@ def _oracle_passing_dev(lay, inp, ref, hkv, d):
 
 @pytest.mark.parametrize("name", list(CASES))
 def test_fused_compress_stage(name):
-    """Scores, top-lp indices and the passing buffer from the one-launch
+    """Scores, top-lp indices and the passing buffer from the fused
     compression against the oracle (indices exact up to near-ties; passing
     rows exact wherever the selection is)."""
     wl, lay, inp, ref = _case(name)
@@ -156,6 +156,26 @@ def test_fused_compress_stage(name):
                 assert np.array_equal(Kn[off:off + e, kv], Kr[off:off + e, kv]), (h, kv)
                 assert np.array_equal(Vn[off:off + e, kv], Vr[off:off + e, kv]), (h, kv)
         off += e
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_fused_compress_scores_equal_the_scoring_stage(name):
+    """Both paths start with the same query-sum kernel and reduce each dot
+    product in the same order, so qsum and the scores agree bit for bit (and
+    with them the selection)."""
+    wl, lay, inp, ref = _case(name)
+    if wl.lp == 0:
+        pytest.skip("lp = 0 compresses nothing")
+    p = spava.Problem.from_workload(wl)
+    d = _dev(inp)
+    qsum_s, scores_s = spava.score(p, d["Q"], d["K"])
+    idx_s = spava.select_topk(p, scores_s)
+    qsum_f, scores_f, idx_f, _, _ = spava.compress(p, d["Q"], d["K"], d["V"])
+    torch.cuda.synchronize()
+    _no_device_error()
+    assert torch.equal(qsum_s, qsum_f)
+    assert torch.equal(scores_s, scores_f)
+    assert torch.equal(idx_s, idx_f)
 
 
 @pytest.mark.parametrize("L,lp,seed", [(5, 2, 0), (1000, 37, 1), (4096, 512, 2), (8191, 1, 3),
@@ -289,7 +309,7 @@ def test_bad_arguments_are_rejected_before_launch():
 
 
 def test_layer_long_block_fallback():
-    """A context block longer than the one-launch compression takes (24576
+    """A context block longer than the fused compression takes (24576
     keys): the layer runs the three stage kernels for steps 1-3 instead, then
     the same attention launch.  Scores and indices are checked in full, rows
     on samples the oracle computes one by one."""
