@@ -94,49 +94,77 @@ __global__ void __cluster_dims__(kQsumSplit, 1, 1) __launch_bounds__(kQsumThread
 }
 
 // ---------------------------------------------------------------------------
-// scores[kv][j] = <qsum[kv], K[key0 + j, kv, :]> for j < nkeys.  K is streamed
-// once with 16-byte loads; the D/8 lanes that hold one (key, head) row reduce
-// with shuffles.  Grid-stride, kScoreUnroll loads in flight per thread.
+// scores[kv][j] = <qsum[kv], K[key0 + j, kv, :]> for j < nkeys.  The rows
+// [key0, key0 + nkeys) of K are one contiguous region (all KV heads); each
+// CTA streams an equal share of it through a ring in shared memory:
+// kScoreSlots 16-byte cp.async copies per thread in flight, each thread
+// reading back only its own cells; the first copies are issued before the
+// wait for the query sum (the kernel is qsum_kernel's programmatic dependent).  The D/8 lanes that hold one (key, head)
+// row reduce with shuffles, in the same order as the fused compression, so
+// both give the same bits.
 // ---------------------------------------------------------------------------
-constexpr int kScoreThreads = 256;
-constexpr int kScoreUnroll = 4;
+constexpr int kScoreThreads = 512;
+constexpr int kScoreSlots = 8;
+constexpr int kScoreChunk = kScoreThreads * 16;   // bytes of one ring slot
+
+__host__ __device__ constexpr int score_smem_bytes(int Hkv, int D) {
+  return kScoreSlots * kScoreChunk + Hkv * D * 4;
+}
 
 template <int D>
-__global__ void __launch_bounds__(kScoreThreads)
+__global__ void __launch_bounds__(kScoreThreads, 2)
     score_kernel(const __nv_bfloat16* __restrict__ K, const float* __restrict__ qsum,
                  float* __restrict__ scores, int64_t key0, int64_t nkeys, int Hkv) {
-  extern __shared__ float sq[];
   constexpr int kParts = D / 8;
-  for (int c = threadIdx.x; c < Hkv * D; c += blockDim.x) sq[c] = qsum[c];
-  __syncthreads();
-  const int64_t cpr = static_cast<int64_t>(Hkv) * kParts;   // chunks per key row
-  const int64_t total = nkeys * cpr;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  extern __shared__ __align__(16) uint8_t dsm[];
+  float* sq = reinterpret_cast<float*>(dsm + kScoreSlots * kScoreChunk);
+  const int tid = threadIdx.x, pc = tid % kParts;
+  const int64_t total = nkeys * Hkv * kParts;   // 16-byte chunks
+  const int64_t items = (total + kScoreThreads - 1) / kScoreThreads;
+  const int64_t it0 = items * blockIdx.x / gridDim.x, it1 = items * (blockIdx.x + 1) / gridDim.x;
+  const int n = static_cast<int>(it1 - it0);
   const uint4* src = reinterpret_cast<const uint4*>(K + key0 * Hkv * D);
-  const int64_t warp_first = static_cast<int64_t>(blockIdx.x) * blockDim.x + (threadIdx.x & ~31);
-  const int lane = threadIdx.x & 31;
-  for (int64_t base = 0; warp_first + base < total; base += stride * kScoreUnroll) {
-    uint4 raw[kScoreUnroll];
-    int64_t ch[kScoreUnroll];
-#pragma unroll
-    for (int u = 0; u < kScoreUnroll; ++u) {
-      ch[u] = warp_first + base + u * stride + lane;
-      raw[u] = ch[u] < total ? __ldcs(src + ch[u]) : make_uint4(0, 0, 0, 0);
+  const uint32_t cell = smem_u32(dsm) + tid * 16;
+  auto issue = [&](int i) {
+    if (i < n) {
+      const int64_t c = (it0 + i) * kScoreThreads + tid;
+      if (c < total) cp_async16(cell + (i % kScoreSlots) * kScoreChunk, src + c);
     }
+    cp_async_commit();
+  };
+  // this thread's (key, head) row, advanced by kScoreThreads / kParts rows per item
+  // without a division per item
+  constexpr int kStep = kScoreThreads / kParts;
+  const int64_t rh0 = (it0 * kScoreThreads + tid) / kParts;
+  int64_t j = rh0 / Hkv;
+  int kv = static_cast<int>(rh0 % Hkv);
+  const int step_j = kStep / Hkv, step_kv = kStep % Hkv;
+#pragma unroll 1
+  for (int i = 0; i < kScoreSlots; ++i) issue(i);
+  grid_dependency_wait();   // launched as qsum_kernel's programmatic dependent
+  for (int c = tid; c < Hkv * D; c += kScoreThreads) sq[c] = __ldcg(qsum + c);
+  __syncthreads();
+#pragma unroll 1
+  for (int i = 0; i < n; ++i) {
+    cp_async_wait<kScoreSlots - 1>();
+    const uint4 raw = ld_shared_v4(cell + (i % kScoreSlots) * kScoreChunk);
+    const __nv_bfloat16* v = reinterpret_cast<const __nv_bfloat16*>(&raw);
+    const float* q = sq + kv * D + pc * 8;
+    float dot = 0.f;
 #pragma unroll
-    for (int u = 0; u < kScoreUnroll; ++u) {
-      const int within = static_cast<int>(ch[u] % cpr);
-      const int kv = within / kParts, pc = within % kParts;
-      const __nv_bfloat16* v = reinterpret_cast<const __nv_bfloat16*>(&raw[u]);
-      const float* q = sq + kv * D + pc * 8;
-      float dot = 0.f;
+    for (int e = 0; e < 8; ++e) dot = fmaf(__bfloat162float(v[e]), q[e], dot);
+    issue(i + kScoreSlots);   // the slot's value is consumed
 #pragma unroll
-      for (int e = 0; e < 8; ++e) dot = fmaf(__bfloat162float(v[e]), q[e], dot);
-#pragma unroll
-      for (int off = kParts / 2; off >= 1; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
-      if (pc == 0 && ch[u] < total) scores[kv * nkeys + ch[u] / cpr] = dot;
+    for (int off = kParts / 2; off >= 1; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+    if (pc == 0 && j < nkeys) scores[kv * nkeys + j] = dot;
+    j += step_j;
+    kv += step_kv;
+    if (kv >= Hkv) {
+      kv -= Hkv;
+      ++j;
     }
   }
+  cp_async_wait<0>();
 }
 
 // ---------------------------------------------------------------------------

@@ -281,23 +281,30 @@ spava_status_t run_score(const Plan& P, const void* Q, const void* K, float* qsu
   else
     qsum_kernel<64><<<qgrid, kQsumThreads, 0, st>>>(q, qsum, P.qs, P.lq, P.Hq, P.G, P.scale);
   if (last_launch() != SPAVA_OK) return SPAVA_ERR_CUDA;
-  const size_t smem = sizeof(float) * P.Hkv * P.d;
-  const int64_t chunks = P.score_cols * P.Hkv * (P.d / 8);
-  int64_t blocks = (chunks + kScoreThreads * kScoreUnroll - 1) / (kScoreThreads * kScoreUnroll);
-  blocks = std::max<int64_t>(1, std::min<int64_t>(blocks, static_cast<int64_t>(sm_count()) * 8));
-  if (P.d == 128) {
-    if (smem > 48 * 1024 &&
-        cudaFuncSetAttribute(score_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-      return SPAVA_ERR_CUDA;
-    score_kernel<128><<<static_cast<unsigned>(blocks), kScoreThreads, smem, st>>>(k, qsum, scores, P.la,
-                                                                                  P.score_cols, P.Hkv);
-  } else {
-    if (smem > 48 * 1024 &&
-        cudaFuncSetAttribute(score_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-      return SPAVA_ERR_CUDA;
-    score_kernel<64><<<static_cast<unsigned>(blocks), kScoreThreads, smem, st>>>(k, qsum, scores, P.la,
-                                                                                 P.score_cols, P.Hkv);
-  }
+  const int smem = score_smem_bytes(P.Hkv, P.d);
+  const int64_t items = (P.score_cols * P.Hkv * (P.d / 8) + kScoreThreads - 1) / kScoreThreads;
+  const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(items, static_cast<int64_t>(sm_count()) * 2));
+  if (cudaFuncSetAttribute(P.d == 128 ? score_kernel<128> : score_kernel<64>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return SPAVA_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+  cfg.blockDim = dim3(kScoreThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const int64_t key0 = P.la, nkeys = P.score_cols;
+  const int hkv = P.Hkv;
+  const cudaError_t e = P.d == 128
+                            ? cudaLaunchKernelEx(&cfg, score_kernel<128>, k, static_cast<const float*>(qsum), scores,
+                                                 key0, nkeys, hkv)
+                            : cudaLaunchKernelEx(&cfg, score_kernel<64>, k, static_cast<const float*>(qsum), scores,
+                                                 key0, nkeys, hkv);
+  if (e != cudaSuccess) return SPAVA_ERR_CUDA;
   return last_launch();
 }
 
