@@ -55,7 +55,7 @@ typedef struct CUstream_st* spava_stream_t;
 typedef enum {
   SPAVA_OK = 0,
   SPAVA_ERR_INVALID_ARG = 1, /* bad shape, null or misaligned pointer       */
-  SPAVA_ERR_UNSUPPORTED = 2, /* valid but outside this build's limits       */
+  SPAVA_ERR_UNSUPPORTED = 2, /* valid but outside this library's limits     */
   SPAVA_ERR_WORKSPACE = 3,   /* workspace missing or smaller than required  */
   SPAVA_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed           */
   SPAVA_ERR_DEVICE = 5       /* a kernel reported a device-side failure     */
