@@ -25,6 +25,8 @@ CASES = {
     "frames_multi": small_workload("frames_multi", 256, (1024,) * 4, 128, 256, 8, 2, 128,
                                    gen="frames"),
     "no_anchor_d64": small_workload("no_anchor_d64", 0, (129, 255, 64, 300, 1, 77), 19, 33, 4, 4, 64),
+    # three KV heads: (row, head) strides and head steps that are not powers of two
+    "kv3_d128": small_workload("kv3_d128", 40, (333, 130, 257, 96), 45, 70, 6, 3, 128),
 }
 
 _cache = {}
