@@ -30,6 +30,9 @@
 //      buffer, so the copy is balanced whatever slices the kept keys fall in.
 // After step 4's barrier no CTA touches another's shared memory, so CTAs
 // leave independently.
+//
+// kSelectOnly: the stage entry spava_select_topk.  Step 1 reads the scores
+// (written by spava_score) instead of computing them, and step 4 is skipped.
 #pragma once
 #include <cooperative_groups.h>
 #include <cuda_bf16.h>
@@ -61,6 +64,8 @@ __host__ __device__ constexpr int compress_slice_cap(int lmax, int nc) {
 __host__ __device__ constexpr int compress_smem_bytes(int lmax, int nc) {
   return kRingBytes + 4 * compress_slice_cap(lmax, nc);
 }
+// The same for the select-only form: no ring.
+__host__ __device__ constexpr int select_smem_bytes(int lmax, int nc) { return 4 * compress_slice_cap(lmax, nc); }
 
 struct CompressParams {
   int32_t start[kMaxV];   // first sequence row of block h
@@ -77,7 +82,7 @@ struct CompressParams {
   int32_t blk[kMaxV];     // the compressed blocks, one per grid row (all h < V-1, or a host mask's)
 };
 
-template <int D>
+template <int D, bool kSelectOnly = false>
 __global__ void __launch_bounds__(kCompressThreads, 2)
     compress_kernel(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restrict__ V,
                     const float* __restrict__ qsum,
@@ -88,7 +93,7 @@ __global__ void __launch_bounds__(kCompressThreads, 2)
   constexpr int kRowsPerIter = kCompressThreads / kParts;  // rows per ring slot
   extern __shared__ __align__(16) uint8_t dsm[];
   const int nc = static_cast<int>(gridDim.x);   // the cluster: one per (block, KV head)
-  uint32_t* keys = reinterpret_cast<uint32_t*>(dsm + kRingBytes);   // [slice] keys, then kept indices
+  uint32_t* keys = reinterpret_cast<uint32_t*>(dsm + (kSelectOnly ? 0 : kRingBytes));   // [slice] keys, then kept indices
   __shared__ uint32_t hx[2][kCompressMaxCtas][256];   // every CTA's counts of a radix pass
   __shared__ uint32_t hist[256], tot[256], low[256];
   __shared__ uint64_t warp_tot[32];
@@ -111,38 +116,43 @@ __global__ void __launch_bounds__(kCompressThreads, 2)
   const int pc = tid % kParts, lr = tid / kParts;
   const uint32_t cell = smem_u32(dsm) + tid * 16;   // this thread's cell of ring slot 0
 
-  // ---- 1. K rows of the slice through the ring; scores and keys
-  const int nItems = (n + kRowsPerIter - 1) / kRowsPerIter;
-  const int64_t row0 = p.start[h] + j0;
-  auto issue = [&](int it) {
-    if (it < nItems) {
-      const int jj = it * kRowsPerIter + lr;
-      if (jj < n) cp_async16(cell + (it % kRingSlots) * kRingChunk, K + ((row0 + jj) * p.Hkv + kv) * D + pc * 8);
-    }
-    cp_async_commit();   // one group per item (empty past the end), so the waits count items
-  };
-#pragma unroll 1
-  for (int it = 0; it < kRingSlots; ++it) issue(it);
-  grid_dependency_wait();   // qsum is complete and visible
-  float q8[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) q8[e] = __ldcg(qsum + kv * D + pc * 8 + e);
   float* srow = scores + static_cast<int64_t>(kv) * p.score_cols + (p.start[h] - p.la) + j0;
+  if constexpr (kSelectOnly) {
+    // ---- 1. this slice's scores into keys
+    for (int i = tid; i < n; i += kCompressThreads) keys[i] = order_key(srow[i]);
+  } else {
+    // ---- 1. K rows of the slice through the ring; scores and keys
+    const int nItems = (n + kRowsPerIter - 1) / kRowsPerIter;
+    const int64_t row0 = p.start[h] + j0;
+    auto issue = [&](int it) {
+      if (it < nItems) {
+        const int jj = it * kRowsPerIter + lr;
+        if (jj < n) cp_async16(cell + (it % kRingSlots) * kRingChunk, K + ((row0 + jj) * p.Hkv + kv) * D + pc * 8);
+      }
+      cp_async_commit();   // one group per item (empty past the end), so the waits count items
+    };
 #pragma unroll 1
-  for (int it = 0; it < nItems; ++it) {
-    cp_async_wait<kRingSlots - 1>();   // this thread's copy of item it has landed
-    const uint4 raw = ld_shared_v4(cell + (it % kRingSlots) * kRingChunk);
-    const __nv_bfloat16* v = reinterpret_cast<const __nv_bfloat16*>(&raw);
-    const int jj = it * kRowsPerIter + lr;
-    float dot = 0.f;
+    for (int it = 0; it < kRingSlots; ++it) issue(it);
+    grid_dependency_wait();   // qsum is complete and visible
+    float q8[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) dot = fmaf(__bfloat162float(v[e]), q8[e], dot);
-    issue(it + kRingSlots);   // the slot's value is consumed
+    for (int e = 0; e < 8; ++e) q8[e] = __ldcg(qsum + kv * D + pc * 8 + e);
+#pragma unroll 1
+    for (int it = 0; it < nItems; ++it) {
+      cp_async_wait<kRingSlots - 1>();   // this thread's copy of item it has landed
+      const uint4 raw = ld_shared_v4(cell + (it % kRingSlots) * kRingChunk);
+      const __nv_bfloat16* v = reinterpret_cast<const __nv_bfloat16*>(&raw);
+      const int jj = it * kRowsPerIter + lr;
+      float dot = 0.f;
 #pragma unroll
-    for (int off = kParts / 2; off >= 1; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
-    if (pc == 0 && jj < n) {
-      srow[jj] = dot;
-      keys[jj] = order_key(dot);
+      for (int e = 0; e < 8; ++e) dot = fmaf(__bfloat162float(v[e]), q8[e], dot);
+      issue(it + kRingSlots);   // the slot's value is consumed
+#pragma unroll
+      for (int off = kParts / 2; off >= 1; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+      if (pc == 0 && jj < n) {
+        srow[jj] = dot;
+        keys[jj] = order_key(dot);
+      }
     }
   }
   __syncthreads();
@@ -265,6 +275,7 @@ __global__ void __launch_bounds__(kCompressThreads, 2)
   if (rank == 0)
     for (int t = kk + tid; t < p.lp; t += kCompressThreads) out[t] = -1;
   cluster.sync();   // the indices of every slice are written; the last access to peer shared memory
+  if constexpr (kSelectOnly) return;
 
   // ---- 4. kept ranks [g0, g1) of the block: K and V rows into the passing buffer
   if (kk > 0) {

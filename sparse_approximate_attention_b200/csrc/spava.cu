@@ -74,8 +74,9 @@ struct DeviceSetup {
   int smem_optin = 227 * 1024;       // largest dynamic + static shared memory of one CTA
   int smem_reserved = 1024;          // shared memory the system reserves per CTA
   int compress_static[2] = {0, 0};   // static shared memory of compress_kernel<64>, <128>
-  // cudaOccupancyMaxActiveClusters of compress_kernel, by (d, nc, dynamic smem)
-  struct ClusterFit { int d, nc, smem, clusters; };
+  int select_static = 0;             // ... of its select-only form
+  // cudaOccupancyMaxActiveClusters of the cluster kernels, by (kernel, nc, dynamic smem)
+  struct ClusterFit { const void* fn; int nc, smem, clusters; };
   std::vector<ClusterFit> compress_fit;
 };
 std::mutex g_setup_mu;
@@ -128,11 +129,15 @@ spava_status_t device_setup(const DeviceSetup** out) {
       s.compress_static[0] = static_cast<int>(fa.sharedSizeBytes);
     if (st == SPAVA_OK && cudaFuncGetAttributes(&fa, compress_kernel<128>) == cudaSuccess)
       s.compress_static[1] = static_cast<int>(fa.sharedSizeBytes);
+    if (st == SPAVA_OK && cudaFuncGetAttributes(&fa, compress_kernel<128, true>) == cudaSuccess)
+      s.select_static = static_cast<int>(fa.sharedSizeBytes);
     if (st == SPAVA_OK &&
         (cudaFuncSetAttribute(compress_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               s.smem_optin - s.compress_static[0]) != cudaSuccess ||
          cudaFuncSetAttribute(compress_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              s.smem_optin - s.compress_static[1]) != cudaSuccess))
+                              s.smem_optin - s.compress_static[1]) != cudaSuccess ||
+         cudaFuncSetAttribute(compress_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              s.smem_optin - s.select_static) != cudaSuccess))
       st = SPAVA_ERR_CUDA;
     s.status = st;
     s.done = true;
@@ -270,6 +275,9 @@ spava_status_t attn_entry(const Plan& P, int tag, const void* Q, const void* K, 
 namespace {
 
 // ----------------------------------------------------------------- stages
+int cluster_fit(const DeviceSetup* ds, const void* fn, int nc, int smem);
+bool compress_params(const Plan& P, CompressParams* cp);
+
 spava_status_t run_score(const Plan& P, const void* Q, const void* K, float* qsum, float* scores,
                          cudaStream_t st) {
   if (!Q || !K || !qsum || !scores || !aligned16(Q) || !aligned16(K)) return SPAVA_ERR_INVALID_ARG;
@@ -308,9 +316,51 @@ spava_status_t run_score(const Plan& P, const void* Q, const void* K, float* qsu
   return last_launch();
 }
 
+// Top-lp of every compressed block.  The cluster select of the fused
+// compression (compress_kernel's select-only form: each CTA holds one slice
+// of the block's scores) when a slice fits in shared memory; else one CTA per
+// (block, KV head) reading the scores from global memory (topk_kernel).
 spava_status_t run_topk(const Plan& P, const float* scores, int32_t* idx, cudaStream_t st) {
   if (P.lp == 0) return SPAVA_OK;
   if (!scores || !idx) return SPAVA_ERR_INVALID_ARG;
+  const DeviceSetup* ds = nullptr;
+  spava_status_t s = device_setup(&ds);
+  if (s != SPAVA_OK) return s;
+  CompressParams cp;
+  if (!compress_params(P, &cp)) return SPAVA_OK;
+  const void* fn = reinterpret_cast<const void*>(compress_kernel<128, true>);
+  const int pairs = P.ncblk * P.Hkv;
+  int nc = 0;
+  for (int c = kCompressMaxCtas; c >= kCompressMinCtas; c /= 2) {   // the first that fits one wave
+    const int b = select_smem_bytes(cp.lmax, c);
+    if (b + ds->select_static <= ds->smem_optin && cluster_fit(ds, fn, c, b) >= pairs) {
+      nc = c;
+      break;
+    }
+  }
+  if (nc == 0 && select_smem_bytes(cp.lmax, kCompressMaxCtas) + ds->select_static <= ds->smem_optin)
+    nc = kCompressMaxCtas;   // more than one wave
+  if (nc > 0) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(nc);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(static_cast<unsigned>(nc), static_cast<unsigned>(P.ncblk), static_cast<unsigned>(P.Hkv));
+    cfg.blockDim = dim3(kCompressThreads);
+    cfg.dynamicSmemBytes = static_cast<size_t>(select_smem_bytes(cp.lmax, nc));
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const __nv_bfloat16* none = nullptr;
+    __nv_bfloat16* none_w = nullptr;
+    const float* no_qsum = nullptr;
+    if (cudaLaunchKernelEx(&cfg, compress_kernel<128, true>, none, none, no_qsum, const_cast<float*>(scores), idx,
+                           none_w, none_w, cp) != cudaSuccess)
+      return SPAVA_ERR_CUDA;
+    return last_launch();
+  }
   TopkParams tp;
   std::memset(&tp, 0, sizeof(tp));
   for (int h = 0; h < P.V - 1; ++h) {
@@ -354,14 +404,15 @@ spava_status_t run_gather(const Plan& P, const void* K, const void* V, const int
   return last_launch();
 }
 
-// Clusters of nc compress_kernel CTAs with `smem` dynamic bytes that can be
-// resident at once (0 when the query fails); cached per device.
-int compress_clusters(const DeviceSetup* ds, int d, int nc, int smem) {
+// Clusters of nc CTAs of the cluster kernel `fn` (compress_kernel in either
+// form) with `smem` dynamic bytes that can be resident at once (0 when the
+// query fails); cached per device.
+int cluster_fit(const DeviceSetup* ds, const void* fn, int nc, int smem) {
   static std::mutex mu;
   std::lock_guard<std::mutex> lock(mu);
   auto& fit = const_cast<DeviceSetup*>(ds)->compress_fit;
   for (const auto& f : fit)
-    if (f.d == d && f.nc == nc && f.smem == smem) return f.clusters;
+    if (f.fn == fn && f.nc == nc && f.smem == smem) return f.clusters;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -374,14 +425,33 @@ int compress_clusters(const DeviceSetup* ds, int d, int nc, int smem) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  const cudaError_t e = d == 128 ? cudaOccupancyMaxActiveClusters(&n, compress_kernel<128>, &cfg)
-                                 : cudaOccupancyMaxActiveClusters(&n, compress_kernel<64>, &cfg);
-  if (e != cudaSuccess) {
+  if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess) {
     cudaGetLastError();   // a failed query is not a launch error
     n = 0;
   }
-  fit.push_back({d, nc, smem, n});
+  fit.push_back({fn, nc, smem, n});
   return n;
+}
+
+// The launch parameters of the cluster kernels for the blocks the plan
+// compresses (all h < V-1, or a host mask's); false when there are none.
+bool compress_params(const Plan& P, CompressParams* cp) {
+  std::memset(cp, 0, sizeof(*cp));
+  for (int h = 0; h < P.V; ++h) {
+    cp->start[h] = P.start[h];
+    cp->L[h] = P.L[h];
+    cp->k[h] = P.lpe[h];
+  }
+  for (int h = 0; h <= P.V; ++h) cp->poff[h] = P.poff[h];
+  cp->Hkv = P.Hkv;
+  cp->lp = P.lp;
+  cp->la = P.la;
+  cp->score_cols = P.score_cols;
+  for (int i = 0; i < P.ncblk; ++i) {
+    cp->blk[i] = P.cblk[i];
+    cp->lmax = std::max(cp->lmax, P.L[P.cblk[i]]);
+  }
+  return P.ncblk > 0;
 }
 
 bool compress_fits(const Plan& P) {
@@ -415,24 +485,9 @@ spava_status_t run_compress(const Plan& P, const void* Q, const void* K, const v
   spava_status_t s = device_setup(&ds);
   if (s != SPAVA_OK) return s;
   CompressParams cp;
-  std::memset(&cp, 0, sizeof(cp));
-  for (int h = 0; h < P.V; ++h) {
-    cp.start[h] = P.start[h];
-    cp.L[h] = P.L[h];
-    cp.k[h] = P.lpe[h];
-  }
-  for (int h = 0; h <= P.V; ++h) cp.poff[h] = P.poff[h];
-  cp.Hkv = P.Hkv;
-  cp.lp = P.lp;
-  cp.la = P.la;
-  cp.score_cols = P.score_cols;
+  if (!compress_params(P, &cp)) return SPAVA_OK;   // a host mask that selects no compressed block
   cp.merge_count = merge_count;
   cp.n_merge = merge_count ? P.n_merge : 0;
-  if (P.ncblk == 0) return SPAVA_OK;   // a host mask that selects no compressed block
-  for (int i = 0; i < P.ncblk; ++i) {
-    cp.blk[i] = P.cblk[i];
-    cp.lmax = std::max(cp.lmax, P.L[P.cblk[i]]);
-  }
   const int pairs = P.ncblk * P.Hkv;
   const int stat = ds->compress_static[P.d == 128 ? 1 : 0];
   // dynamic bytes above which two CTAs (dynamic + static + what the system
@@ -444,7 +499,9 @@ spava_status_t run_compress(const Plan& P, const void* Q, const void* K, const v
     int b = compress_smem_bytes(cp.lmax, sh.nc);
     if (sh.spread) b = std::max(b, spread);
     if (b + stat > ds->smem_optin) continue;
-    if (compress_clusters(ds, P.d, sh.nc, b) >= pairs) {
+    const void* fn = P.d == 128 ? reinterpret_cast<const void*>(compress_kernel<128>)
+                                : reinterpret_cast<const void*>(compress_kernel<64>);
+    if (cluster_fit(ds, fn, sh.nc, b) >= pairs) {
       nc = sh.nc;
       smem = b;
       break;
