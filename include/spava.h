@@ -152,7 +152,9 @@ spava_status_t spava_score_variant(const spava_problem_t* prob, const void* Q,
 /* Step 2, top-lp per block and KV head ([PR] "What carries the argument":
  * each context block compressed to its top-lp key-value pairs).  Larger
  * score first; equal scores keep the lower index; -0.0 equals +0.0.
- * Writes `idx` (ascending, -1 padded). */
+ * Writes `idx` (ascending, -1 padded).  One cluster of CTAs per (block, KV
+ * head) selects across its slices of the scores (the fused compression's
+ * select); blocks too long for that use one CTA each. */
 spava_status_t spava_select_topk(const spava_problem_t* prob,
                                  const float* scores, int32_t* idx,
                                  spava_stream_t stream);
