@@ -137,7 +137,11 @@ spava_status_t device_setup(const DeviceSetup** out) {
          cudaFuncSetAttribute(compress_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               s.smem_optin - s.compress_static[1]) != cudaSuccess ||
          cudaFuncSetAttribute(compress_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              s.smem_optin - s.select_static) != cudaSuccess))
+                              s.smem_optin - s.select_static) != cudaSuccess ||
+         cudaFuncSetAttribute(score_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, s.smem_optin) !=
+             cudaSuccess ||
+         cudaFuncSetAttribute(score_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, s.smem_optin) !=
+             cudaSuccess))
       st = SPAVA_ERR_CUDA;
     s.status = st;
     s.done = true;
@@ -281,6 +285,11 @@ bool compress_params(const Plan& P, CompressParams* cp);
 spava_status_t run_score(const Plan& P, const void* Q, const void* K, float* qsum, float* scores,
                          cudaStream_t st) {
   if (!Q || !K || !qsum || !scores || !aligned16(Q) || !aligned16(K)) return SPAVA_ERR_INVALID_ARG;
+  const DeviceSetup* ds = nullptr;
+  spava_status_t s = device_setup(&ds);
+  if (s != SPAVA_OK) return s;
+  const int smem = score_smem_bytes(P.Hkv, P.d);   // the ring + the query sums of every KV head
+  if (smem > ds->smem_optin) return SPAVA_ERR_UNSUPPORTED;
   const auto* q = static_cast<const __nv_bfloat16*>(Q);
   const auto* k = static_cast<const __nv_bfloat16*>(K);
   dim3 qgrid(kQsumSplit, P.Hkv);
@@ -289,12 +298,8 @@ spava_status_t run_score(const Plan& P, const void* Q, const void* K, float* qsu
   else
     qsum_kernel<64><<<qgrid, kQsumThreads, 0, st>>>(q, qsum, P.qs, P.lq, P.Hq, P.G, P.scale);
   if (last_launch() != SPAVA_OK) return SPAVA_ERR_CUDA;
-  const int smem = score_smem_bytes(P.Hkv, P.d);
   const int64_t items = (P.score_cols * P.Hkv * (P.d / 8) + kScoreThreads - 1) / kScoreThreads;
-  const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(items, static_cast<int64_t>(sm_count()) * 2));
-  if (cudaFuncSetAttribute(P.d == 128 ? score_kernel<128> : score_kernel<64>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-    return SPAVA_ERR_CUDA;
+  const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(items, static_cast<int64_t>(ds->sm_count) * 2));
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
