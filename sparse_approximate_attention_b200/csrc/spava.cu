@@ -434,6 +434,7 @@ int cluster_fit(const DeviceSetup* ds, const void* fn, int nc, int smem) {
     cudaGetLastError();   // a failed query is not a launch error
     n = 0;
   }
+  if (fit.size() >= 256) fit.clear();   // the key includes the block length: bound the cache
   fit.push_back({fn, nc, smem, n});
   return n;
 }
