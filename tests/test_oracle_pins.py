@@ -439,3 +439,78 @@ def test_selection_overlap_bounds():
     comp = {h: np.stack([np.setdiff1d(np.arange(lay.block_lens[h]), a[h][kv])[:lay.lp_eff(h)]
                          for kv in range(lay.num_kv_heads)]) for h in a}
     assert oracle.selection_overlap(lay, a, comp) == 0.0
+
+
+# ------------------------------------------------ random layouts, whole layer
+from hypothesis import HealthCheck, given, settings, strategies as st  # noqa: E402
+
+
+@st.composite
+def _layouts(draw):
+    H = draw(st.integers(1, 3))
+    blocks = draw(st.lists(st.integers(1, 40), min_size=2 * H, max_size=2 * H))
+    la = draw(st.integers(0, 20))
+    lq = draw(st.integers(1, 12))
+    lp = draw(st.integers(0, 45))
+    hq, hkv = draw(st.sampled_from([(1, 1), (2, 1), (4, 2), (6, 3), (4, 4)]))
+    d = draw(st.sampled_from([8, 16]))
+    seed = draw(st.integers(0, 10_000))
+    return H, blocks, la, lq, lp, hq, hkv, d, seed
+
+
+@settings(max_examples=40, deadline=None, derandomize=True, suppress_health_check=[HealthCheck.too_slow])
+@given(_layouts())
+def test_layer_random_layouts_against_masked_sdpa(case):
+    """Every output row of random tiny layouts against library attention with
+    an explicit boolean mask built here from the pages' key lists: anchor rows
+    causal over A; context rows of host h over A, the top-lp_eff keys of every
+    earlier block (chosen by torch.topk on the full Q_qr K^T matrix summed over
+    the query rows and the KV group's heads) and B^(h) causally; query rows
+    dense causal.  Covers blocks of one key, lp above the block length, la = 0,
+    lp = 0 and GQA groups of 1-3 heads."""
+    H, blocks, la, lq, lp, hq, hkv, d, seed = case
+    lay = oracle.make_layout(H, la, blocks, lq, lp, hq, hkv, d)
+    g = torch.Generator().manual_seed(seed)
+    n = lay.n
+    Q = torch.randn(n, hq, d, generator=g, dtype=torch.float64)
+    K = torch.randn(n, hkv, d, generator=g, dtype=torch.float64)
+    Vv = torch.randn(n, hkv, d, generator=g, dtype=torch.float64)
+    out = oracle.layer_fwd(lay, Q, K, Vv)
+    G, qs, starts = hq // hkv, lay.query_start, lay.block_starts
+    masks = []
+    for kv in range(hkv):
+        Qg = Q[qs:qs + lq, kv * G:(kv + 1) * G]                       # [lq, G, d]
+        m = torch.zeros(n, n, dtype=torch.bool)
+        for r in range(la):
+            m[r, :r + 1] = True
+        passing = []
+        for h in range(2 * H):
+            s0, L = starts[h], blocks[h]
+            for r in range(s0, s0 + L):
+                m[r, :la] = True
+                m[r, s0:r + 1] = True
+                for c in passing:
+                    m[r, c] = True
+            e = min(lp, L)
+            if h < 2 * H - 1 and e > 0:
+                logits = lay.scale * torch.einsum("igc,jc->igj", Qg, K[s0:s0 + L, kv])
+                s = logits.sum(dim=(0, 1))                             # [L]
+                top = torch.topk(s, e, sorted=True)
+                if e < L:   # a near-tie at the boundary has no unique answer
+                    rest = torch.topk(s, e + 1, sorted=True).values[-1]
+                    if abs(float(top.values[-1] - rest)) <= 1e-9 * float(s.abs().max()):
+                        return
+                chosen = sorted(int(j) for j in top.indices)
+                assert list(out["idx"][h][kv][:e]) == chosen, (h, kv)
+                passing += [s0 + j for j in chosen]
+        for r in range(qs, n):
+            m[r, :r + 1] = True
+        masks.append(m)
+    for head in range(hq):
+        m = masks[head // G]
+        q, k, v = Q[:, head], K[:, head // G], Vv[:, head // G]
+        o = F.scaled_dot_product_attention(q[None, None], k[None, None], v[None, None], attn_mask=m[None, None],
+                                           scale=lay.scale)[0, 0]
+        z = (lay.scale * (q @ k.T)).masked_fill(~m, -math.inf)
+        np.testing.assert_allclose(out["O"][:, head], o.numpy(), atol=1e-11)
+        np.testing.assert_allclose(out["lse"][head], torch.logsumexp(z, dim=-1).numpy(), atol=1e-11)
